@@ -1,0 +1,549 @@
+"""Benchmark of the paged decode path (copy-on-write block copy + kv_append +
+paged decode attention) on B200, one JSON line on stdout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload KEY]
+                    [--block-size B] [--partition P] [--impl ours|reference]
+
+A step is one pass of the whole path over one batch: block_copy of the
+batch's copy-on-write pairs (every layer), then for each layer kv_append of
+one new token per sequence and paged decode attention.  Inputs are seeded
+synthetic data of the workload's shapes (``workload/``), resident in HBM
+before the timed region; L2 reuse across steps is prevented by rotating
+through several copies of the KV pools whose total is over 4x the L2 size.
+
+Multi-GPU (torchrun): every rank runs its own independent batch (weak
+scaling, no data-path collective); the timed region is bracketed by a barrier
+and the device time is the max over ranks.
+"""
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workload import make_workload, rank_seed  # noqa: E402
+from workload.configs import get_spec  # noqa: E402
+
+METRIC = "paged decode attention KV GB/s and % of HBM peak; decode tokens/s per layer"
+UNIT = "GB/s"
+DEFAULT_WORKLOAD = "continuous_batch"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "attention_traffic.json")
+KERNEL_SOURCES = ["pkv_device.cuh", "paged_attention.cuh", "pagedkv.cu"]
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_cache_378_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_traffic(workload_key, block_size):
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    if absent, for another workload, or taken on different kernel source."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    for r in rec.get("captures", []):
+        if r.get("workload") == workload_key and int(r.get("block_size", -1)) == block_size \
+                and r.get("kernel_source_hash") == kernel_source_hash():
+            return r.get("dram_bytes_per_launch")
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons in the background."""
+
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, pci_bus_id=None, period_ms=100):
+        self.pci = (pci_bus_id or "").lower()
+        self.period_ms = period_ms
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms={self.period_ms}"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except OSError:
+            self.proc = None
+            return self
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            if self.pci and not parts[1].lower().endswith(self.pci[-12:]):
+                continue
+            self.rows.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        rows = [r for t, r in self.rows if t0 <= t <= t1]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        mx = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((num(r[4]) or 0.0) for r in rows)}
+
+
+def pci_bus_id(dev):
+    try:
+        from cuda.bindings import runtime as rt
+        err, bus = rt.cudaDeviceGetPCIBusId(32, dev)
+        if int(err) == 0:
+            return bus.decode().rstrip("\x00") if isinstance(bus, bytes) else str(bus)
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+# the GPU step through the C ABI
+# ---------------------------------------------------------------------------
+
+class GpuStep:
+    """One decode step through the C ABI with arguments marshalled once.
+
+    Calls the library's entry points directly (the same C functions the
+    Python binding wraps), so per-step host overhead stays far below the
+    device time of a step.
+    """
+
+    def __init__(self, pkv, w, replicas, partition, device):
+        from paged_kv_cache_378_b200._lib import PkvCache
+        self.lib = pkv.library()
+        spec = w.spec
+        self.w = w
+        self.L = spec.num_layers
+        self.N = w.num_seqs
+        self.Hq = spec.num_q_heads
+        self.device = device
+        self.stream = torch.cuda.current_stream(device)
+        self.sp = ctypes.c_void_p(self.stream.cuda_stream)
+        self.replicas = replicas
+        self.caches = []
+        L, NB, H, B, D = w.k_pool.shape
+        for kp, vp in replicas:
+            c = PkvCache(kp.data_ptr(), vp.data_ptr(), L, NB, H, B, D)
+            self.caches.append((c, ctypes.byref(c)))
+        self.q = w.q
+        self.k_new, self.v_new = w.k_new, w.v_new
+        self.tables = torch.from_numpy(w.block_tables).to(device)
+        self.lens = torch.from_numpy(w.seq_lens).to(device)
+        self.slots = torch.from_numpy(w.slot_mapping).to(device)
+        self.pairs = torch.from_numpy(w.copy_pairs).to(device)
+        self.npairs = int(w.copy_pairs.shape[0])
+        self.out = torch.empty_like(w.q)
+        self.partition = int(partition)
+        self.ws = pkv.make_workspace(self.N, self.Hq, H, D, w.max_blocks, B, self.partition,
+                                     device=device)
+        self.scale = ctypes.c_float(spec.scale)
+        self.maxb = w.max_blocks
+        self.launches_per_step = (1 if self.npairs else 0) + 2 * self.L
+
+    def run(self, step_index, evl=None):
+        """Launch one step; ``evl`` = per-layer (start, end) events around attention."""
+        lib = self.lib
+        _, cref = self.caches[step_index % len(self.caches)]
+        rc = 0
+        if self.npairs:
+            rc |= lib.pkv_block_copy(cref, self.pairs.data_ptr(), self.npairs, self.sp)
+        for layer in range(self.L):
+            rc |= lib.pkv_kv_append(cref, layer, self.k_new[layer].data_ptr(),
+                                    self.v_new[layer].data_ptr(), self.slots.data_ptr(), self.N,
+                                    self.sp)
+            if evl is not None:
+                evl[layer][0].record(self.stream)
+            rc |= lib.pkv_paged_decode_attention(
+                cref, layer, self.q[layer].data_ptr(), self.N, self.Hq, self.tables.data_ptr(),
+                self.maxb, self.lens.data_ptr(), self.scale, self.out[layer].data_ptr(),
+                self.ws.data_ptr(), self.ws.numel(), self.partition, self.sp)
+            if evl is not None:
+                evl[layer][1].record(self.stream)
+        if rc:
+            raise RuntimeError(f"pagedkv call failed (status {rc})")
+
+
+def e2e_run(pkv, w, gs, steps, device):
+    """Same step through the C ABI with host buffers: per step, H2D of the
+    step's inputs from pinned memory and D2H of the attention output."""
+    host = dict(q=w.q.cpu().pin_memory(), k_new=w.k_new.cpu().pin_memory(),
+                v_new=w.v_new.cpu().pin_memory(),
+                tables=torch.from_numpy(w.block_tables).pin_memory(),
+                lens=torch.from_numpy(w.seq_lens).pin_memory(),
+                slots=torch.from_numpy(w.slot_mapping).pin_memory(),
+                pairs=torch.from_numpy(w.copy_pairs).pin_memory())
+    out_host = torch.empty(gs.out.shape, dtype=gs.out.dtype).pin_memory()
+    dev_bufs = dict(q=gs.q, k_new=gs.k_new, v_new=gs.v_new, tables=gs.tables, lens=gs.lens,
+                    slots=gs.slots, pairs=gs.pairs)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    s = gs.stream
+
+    def one(i):
+        for k, t in host.items():
+            dev_bufs[k].copy_(t, non_blocking=True)
+        gs.run(i)
+        out_host.copy_(gs.out, non_blocking=True)
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for i in range(steps):
+        one(i)
+    e1.record(s)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+
+def _u16(t):
+    return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def oracle_full_step(oa, w, host):
+    """The oracle's whole step on every sequence: copies, append, attention."""
+    L = w.spec.num_layers
+    kp, vp = oa.block_copy(host["k"], host["v"], w.copy_pairs)
+    for layer in range(L):
+        k2, v2 = oa.kv_append(kp[layer], vp[layer], host["k_new"][layer], host["v_new"][layer],
+                              w.slot_mapping, w.block_size)
+        oa.paged_decode_attention(host["q"][layer], k2, v2, w.block_tables, w.seq_lens,
+                                  w.block_size, w.spec.scale)
+
+
+def cpu_threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([1] + [int(i.get("num_threads", 1)) for i in threadpool_info()])
+    except Exception:
+        return 1
+
+
+def limit_blas_threads():
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(1)
+    except Exception:
+        return None
+
+
+def host_workload(key, block_size, seed):
+    w = make_workload(key, block_size=block_size, seed=seed, device="cpu", poison=False)
+    host = dict(k=_u16(w.k_pool), v=_u16(w.v_pool), q=_u16(w.q), k_new=_u16(w.k_new),
+                v_new=_u16(w.v_new))
+    return w, host
+
+
+def cpu_baseline(key, block_size, seed, unique_bytes, min_seconds=10.0):
+    from oracle import attention as oa
+    lim = limit_blas_threads()
+    w, host = host_workload(key, block_size, seed)
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle_full_step(oa, w, host)
+        n += 1
+        if time.perf_counter() - t0 >= min_seconds:
+            break
+    dt = (time.perf_counter() - t0) / n
+    cores = cpu_threads_used() if lim is None else 1
+    return {"value": unique_bytes * w.spec.num_layers / dt / 1e9, "unit": UNIT, "cores": cores,
+            "kind": "oracle",
+            "sample": f"the whole step of this workload (all {w.num_seqs} sequences: block_copy, "
+                      f"kv_append, attention, {w.spec.num_layers} layer(s)), repeated {n}x, "
+                      f"{dt:.2f} s per step, numpy fp64, 1 thread"}
+
+
+def run_reference(args):
+    """--impl reference: the oracle timed as it stands on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from oracle import attention as oa
+    spec = get_spec(args.workload)
+    B = args.block_size or spec.block_size
+    lim = limit_blas_threads()
+    w, host = host_workload(args.workload, B, spec.seed)
+    kp, vp = oa.block_copy(host["k"], host["v"], w.copy_pairs)
+    k2, v2 = oa.kv_append(kp[0], vp[0], host["k_new"][0], host["v_new"][0], w.slot_mapping,
+                          w.block_size)
+    per_seq_bytes = w.seq_lens.astype(np.int64) * 2 * spec.num_kv_heads * spec.head_dim * 2
+    # calibrate: seconds per KV byte of the oracle's attention
+    cal = list(range(0, w.num_seqs, max(1, w.num_seqs // 8)))
+    t = time.perf_counter()
+    oa.paged_decode_attention(host["q"][0][cal], k2, v2, w.block_tables[cal], w.seq_lens[cal],
+                              w.block_size, spec.scale)
+    s_per_byte = (time.perf_counter() - t) / max(1, int(per_seq_bytes[cal].sum()))
+    budget = 120.0 / (args.steps + args.warmup)
+    target = budget / s_per_byte
+    m = int(np.clip(np.searchsorted(np.cumsum(per_seq_bytes), target), 1, w.num_seqs))
+
+    def step(i):
+        idx = [(i * m + j) % w.num_seqs for j in range(m)]
+        oa.paged_decode_attention(host["q"][0][idx], k2, v2, w.block_tables[idx], w.seq_lens[idx],
+                                  w.block_size, spec.scale)
+        return int(per_seq_bytes[idx].sum())
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    tot = 0
+    for i in range(args.steps):
+        tot += step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    val = tot / dt / 1e9
+    cores = 1 if lim is not None else cpu_threads_used()
+    sample = (f"attention of {m} of {w.num_seqs} sequences per step (round robin), layer 0, after "
+              f"the oracle's block_copy and kv_append of the step; numpy fp64")
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT,
+            "n_gpus": int(os.environ.get("WORLD_SIZE", args.gpus)), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "block_size": B},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# main (our arm)
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--block-size", type=int, default=0)
+    ap.add_argument("--partition", type=int, default=-1, help="-1: the workload's, 0: library default")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--soak-seconds", type=float, default=1.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=device)
+
+    import paged_kv_cache_378_b200 as pkv
+
+    spec = get_spec(args.workload)
+    B = args.block_size or spec.block_size
+    part = spec.partition_tokens if args.partition < 0 else args.partition
+    seed = rank_seed(spec.seed, rank)
+
+    # cpu baseline first, before the GPU is busy (rank 0 at N = 1 only)
+    w_meta = make_workload(args.workload, block_size=B, seed=seed, values=False)
+    unique_bytes = w_meta.unique_kv_bytes_read()
+    logical_bytes = w_meta.kv_bytes_read()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, B, seed, unique_bytes)
+
+    w = make_workload(args.workload, block_size=B, seed=seed, device=device, poison=False)
+    pool_bytes = 2 * w.k_pool.numel() * w.k_pool.element_size()
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    nrep = max(1, min(16, math.ceil(4 * l2 / pool_bytes)))
+    replicas = [(w.k_pool, w.v_pool)] + [(w.k_pool.clone(), w.v_pool.clone()) for _ in range(nrep - 1)]
+    gs = GpuStep(pkv, w, replicas, part, device)
+    pkv.get_device_status(reset=True)
+
+    # warm-up
+    for i in range(args.warmup):
+        gs.run(i)
+    torch.cuda.synchronize(device)
+    if pkv.get_device_status(reset=True):
+        raise SystemExit("device status raised during warm-up")
+
+    sampler = ClockSampler(pci_bus_id(local)).start()
+    time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps * spec.num_layers)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    wall0 = time.time()
+    t_start.record(gs.stream)
+    nl = spec.num_layers
+    for i in range(args.steps):
+        gs.run(i, evs[i * nl:(i + 1) * nl])
+    t_end.record(gs.stream)
+    torch.cuda.synchronize(device)
+    wall1 = time.time()
+    if dist is not None:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+    soak_until = wall1
+    if wall1 - wall0 < args.soak_seconds:      # keep the GPU busy so the clock sampler sees load
+        i = args.steps
+        while time.time() - wall0 < args.soak_seconds:
+            for _ in range(50):
+                gs.run(i)
+                i += 1
+            torch.cuda.synchronize(device)
+        soak_until = time.time()
+    sampler.stop()
+    clocks = sampler.summary(wall0 - 0.05, soak_until + 0.05)
+    clocks["window"] = "timed region" if soak_until == wall1 else "timed region + untimed soak"
+    status = pkv.get_device_status(reset=True)
+    if status:
+        raise SystemExit(f"device status {status:#x} raised in the timed region")
+
+    attn_ms = [a.elapsed_time(b) for a, b in evs]
+    attn_avg_ms = sum(attn_ms) / len(attn_ms)
+
+    # totals over ranks
+    ms_max = ms
+    bytes_total = unique_bytes * spec.num_layers
+    seqs_total = w.num_seqs
+    if dist is not None:
+        t = torch.tensor([ms, bytes_total, seqs_total], dtype=torch.float64, device=device)
+        tm = t.clone()
+        dist.all_reduce(tm[0:1], op=dist.ReduceOp.MAX)
+        dist.all_reduce(tm[1:3], op=dist.ReduceOp.SUM)
+        ms_max, bytes_total, seqs_total = float(tm[0]), float(tm[1]), float(tm[2])
+    ms_per_step = ms_max / args.steps
+    value = bytes_total / (ms_per_step * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = e2e_run(pkv, w, gs, args.e2e_steps, device)
+        if dist is not None:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t[0])
+        e2e = {"value": bytes_total / (e_ms * 1e-3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e_ms, "steps": args.e2e_steps}
+
+    peak, peak_kind = load_peak()
+    q_out_bytes = 2 * w.num_seqs * spec.num_q_heads * spec.head_dim * 2
+    meta_bytes = w.block_tables.nbytes + w.seq_lens.nbytes
+    alg_bytes = unique_bytes + q_out_bytes + meta_bytes
+    achieved = alg_bytes / (attn_avg_ms * 1e-3) / 1e9
+    traffic = load_traffic(args.workload, B)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "title": spec.title, "num_seqs": w.num_seqs,
+                   "num_layers": spec.num_layers, "q_heads": spec.num_q_heads,
+                   "kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim, "block_size": B,
+                   "partition_tokens": pkv.partition_tokens(w.num_seqs, spec.num_kv_heads,
+                                                            spec.head_dim, w.max_blocks, B, part),
+                   "l2": f"inputs larger than L2: {nrep} rotating copies of the KV pools, "
+                         f"{nrep * pool_bytes / 1e9:.2f} GB vs {l2 / 1e6:.0f} MB L2",
+                   "parallelism": f"dp{world} (independent batches, no collective)"},
+        "pct_hbm_peak": 100.0 * value / peak,
+        "decode_tokens_per_s_per_layer": seqs_total / (ms_per_step * 1e-3),
+        "kv_bytes_per_step": {"unique": unique_bytes * spec.num_layers,
+                              "logical": logical_bytes * spec.num_layers},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "paged_attention_kernel", "alg_bytes_per_launch": alg_bytes,
+                     "avg_launch_us": attn_avg_ms * 1e3, "peak_source": f"{peak_kind} hbm_gbs"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": gs.launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

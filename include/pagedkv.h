@@ -1,0 +1,205 @@
+/*
+ * pagedkv.h -- C ABI of the paged KV-cache decode path (sm_100a).
+ *
+ * Three operations, each one asynchronous launch sequence on the caller's
+ * CUDA stream:
+ *
+ *   pkv_block_copy              copy-on-write of shared tail blocks
+ *   pkv_kv_append               store each new token's K and V in its slot
+ *   pkv_paged_decode_attention  decode attention read through block tables
+ *
+ * Sources: "Infra: PagedAttention" (Fanyi Pu), sections "按 Block 分配" and
+ * "共享前缀，分叉时 Copy-on-write"; ithelp.ithome.com.tw article 10405755,
+ * sections "PagedAttention 的核心想法" and "手動畫一次 block table".
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every pointer argument except `cache` (host) and `status_out` (host) is
+ *    a DEVICE pointer on the current device, owned by the caller.  The
+ *    library never allocates, frees or keeps a pointer past the call.
+ *  - bf16 buffers (pools, q, k_new, v_new, out) must be 16-byte aligned;
+ *    the pools, q and out are dense row-major as documented per argument.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls return before the GPU work finishes; nothing inside a
+ *    call synchronises the host.
+ *  - Return value: PKV_OK, or a negative PKV_ERR_* code when an argument
+ *    check fails on the host (nothing is launched) or a launch fails.
+ *  - Faults found by the kernels themselves (a block id or slot outside the
+ *    pool, a sequence longer than its table, a bounded wait that gave up)
+ *    never trap: the kernel skips the access and ORs a PKV_DEV_* bit into a
+ *    per-device status word read by pkv_get_device_status().  Outputs of a
+ *    launch that raised a device bit are undefined.
+ *
+ * KV cache layout (the pages fix none; this is the library's contract)
+ * ------------------------------------------------------------------
+ *   k_pool, v_pool : bf16 [num_layers][num_blocks][num_kv_heads][block_size][head_dim]
+ * The tile of one (physical block, kv head) is contiguous
+ * (block_size * head_dim * 2 bytes).  Slot s (flat numbering) is token row
+ * s % block_size of physical block s / block_size, as in the page's example:
+ * with table [3, 0, 4] and B = 4, position 8 is logical block 2 -> P4, row 0.
+ *
+ * Supported shapes: head_dim in {64, 128}; block_size in {8, 16, 32};
+ * num_q_heads = G * num_kv_heads with G in {1, 2, 4, 8}.  Query head h
+ * reads kv head h / G (contiguous GQA groups).
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PKV_ABI_VERSION 1
+
+/* host-side status codes */
+#define PKV_OK                0
+#define PKV_ERR_NULL         -1  /* a required pointer is NULL */
+#define PKV_ERR_SHAPE        -2  /* a size is negative or inconsistent */
+#define PKV_ERR_ALIGN        -3  /* a bf16 buffer is not 16-byte aligned */
+#define PKV_ERR_WORKSPACE    -4  /* workspace missing or too small */
+#define PKV_ERR_UNSUPPORTED  -5  /* head_dim / block_size / group size not built */
+#define PKV_ERR_CUDA         -6  /* a CUDA runtime call or launch failed */
+#define PKV_ERR_LAYER        -7  /* layer index outside [0, num_layers) */
+
+/* device-side status bits (pkv_get_device_status) */
+#define PKV_DEV_RANGE    0x1u  /* block id or slot outside the pool: access skipped */
+#define PKV_DEV_LENGTH   0x2u  /* seq_len above max_blocks_per_seq * block_size: clamped */
+#define PKV_DEV_TIMEOUT  0x4u  /* a bounded wait for staged KV gave up */
+
+typedef struct pkv_cache {
+    void*   k_pool;        /* bf16 [num_layers][num_blocks][num_kv_heads][block_size][head_dim] */
+    void*   v_pool;        /* same shape as k_pool */
+    int32_t num_layers;
+    int32_t num_blocks;
+    int32_t num_kv_heads;
+    int32_t block_size;
+    int32_t head_dim;
+} pkv_cache_t;
+
+/*
+ * pkv_kv_append -- write the K and V of `num_tokens` new tokens into their slots.
+ *
+ * Defines: a new token fills the next free slot of its sequence's tail block
+ * (the caller's block manager picks the slot: a fresh block only once the
+ * tail is full) -- ithelp article 10405755, "手動畫一次 block table";
+ * "Infra: PagedAttention", "按 Block 分配".
+ *
+ *   layer         layer of the pools to write, 0 <= layer < num_layers
+ *   k_new, v_new  bf16 [num_tokens][num_kv_heads][head_dim]
+ *   slot_mapping  int64 [num_tokens]; slot < 0 means padding (skipped);
+ *                 slot >= num_blocks*block_size sets PKV_DEV_RANGE (skipped)
+ *   num_tokens    >= 0; 0 launches nothing
+ * The bf16 bit patterns are moved unchanged (NaN payloads and -0 survive).
+ * Precondition: no slot appears twice (the later write would race).
+ */
+int pkv_kv_append(const pkv_cache_t* cache, int layer,
+                  const void* k_new, const void* v_new,
+                  const int64_t* slot_mapping, int num_tokens, void* stream);
+
+/*
+ * pkv_block_copy -- copy whole physical blocks, every layer, K and V.
+ *
+ * Defines: copy-on-write of a shared, partially filled tail block: before a
+ * writer appends to a block whose reference count is above one, the block is
+ * copied and the writer remapped to the copy; full prefix blocks stay shared
+ * -- "Infra: PagedAttention", "共享前缀，分叉时 Copy-on-write" and its figure
+ * (A copies P0 -> P4, B keeps P0, P3 stays shared).
+ *
+ *   src_dst_pairs  int32 [num_pairs][2] = (src block, dst block)
+ *   num_pairs      >= 0; 0 launches nothing
+ * For every pair and every layer l: pool[l][dst] = pool[l][src] (all heads,
+ * all rows, K and V), bit exact.  A block id outside [0, num_blocks) sets
+ * PKV_DEV_RANGE and that pair is skipped.  Precondition: dst ids are
+ * distinct and none is also a src (otherwise the copies race).
+ */
+int pkv_block_copy(const pkv_cache_t* cache, const int32_t* src_dst_pairs,
+                   int num_pairs, void* stream);
+
+/*
+ * pkv_attention_workspace_bytes -- bytes of workspace pkv_paged_decode_attention
+ * needs for these sizes (split-K partials plus one counter per (sequence,
+ * kv head)).  `partition_tokens` as passed to the attention call (0 = the
+ * library's choice).  Returns 0 for invalid sizes.
+ */
+size_t pkv_attention_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,
+                                     int head_dim, int max_blocks_per_seq, int block_size,
+                                     int partition_tokens);
+
+/*
+ * pkv_partition_tokens -- the KV partition length (tokens) the attention call
+ * uses for these sizes; `requested` 0 picks the library's default, otherwise
+ * it is rounded up to the kernel's tile (16 tokens, or the block size when
+ * larger).  Returns <= 0 for invalid sizes.
+ */
+int pkv_partition_tokens(int num_seqs, int num_kv_heads, int head_dim,
+                         int max_blocks_per_seq, int block_size, int requested);
+
+/*
+ * pkv_workspace_init -- zero a workspace before its first use (asynchronous
+ * memset on `stream`).  The attention kernel leaves every counter back at
+ * zero when it finishes, so a workspace is initialised once, not per call.
+ */
+int pkv_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * pkv_paged_decode_attention -- one decode step of attention for `num_seqs`
+ * sequences, reading K and V through block tables.
+ *
+ * Defines: the attention formula is unchanged by paging; the kernel looks up
+ * the block table and reads the physical blocks in place, without copying
+ * them into one contiguous range (ithelp article 10405755, "PagedAttention
+ * 的核心想法"; "Infra: PagedAttention", "按 Block 分配").  Score
+ * s_i = scale * q . k_i, softmax over every visible token.  Long sequences
+ * are split into partitions of `partition_tokens` tokens; each partition
+ * keeps (max score m_r, Z_r = sum e^{s_i - m_r}, unnormalised output) and the
+ * partitions are merged with o = sum_r e^{m_r - M} Z_r o_r / sum_r e^{m_r - M} Z_r,
+ * M = max_r m_r ("Infra: PagedAttention", "按 Block 分配", the merge
+ * equation and the paragraph on max rescaling).
+ *
+ *   layer              layer of the pools to read
+ *   q                  bf16 [num_seqs][num_q_heads][head_dim]
+ *   block_tables       int32 [num_seqs][max_blocks_per_seq]; entry j of
+ *                      sequence s is the physical block of positions
+ *                      [j*B, (j+1)*B); entries past ceil(len/B) are never read
+ *   seq_lens           int32 [num_seqs], tokens to attend to (including a
+ *                      token appended this step); 0 gives a zero output;
+ *                      values above max_blocks_per_seq*B set PKV_DEV_LENGTH
+ *                      and are clamped
+ *   scale              score scale, usually 1/sqrt(head_dim)
+ *   out                bf16 [num_seqs][num_q_heads][head_dim], round to
+ *                      nearest even from fp32
+ *   workspace          device buffer of at least
+ *                      pkv_attention_workspace_bytes(...) bytes, 16-byte
+ *                      aligned, zeroed once (pkv_workspace_init) before its
+ *                      first use; may be NULL only if every sequence fits in
+ *                      one partition (max_blocks_per_seq*B <= partition)
+ *   partition_tokens   0 = library default, else the split-K partition length
+ * Concurrent calls must not share a workspace.
+ */
+int pkv_paged_decode_attention(const pkv_cache_t* cache, int layer,
+                               const void* q, int num_seqs, int num_q_heads,
+                               const int32_t* block_tables, int max_blocks_per_seq,
+                               const int32_t* seq_lens, float scale, void* out,
+                               void* workspace, size_t workspace_bytes,
+                               int partition_tokens, void* stream);
+
+/*
+ * pkv_get_device_status -- read (and with reset != 0, clear) the device status
+ * word of the current device.  Synchronises the device first.
+ */
+int pkv_get_device_status(unsigned int* status_out, int reset);
+
+/* pkv_strerror -- static text for a PKV_ERR_* code. */
+const char* pkv_strerror(int code);
+
+/* pkv_abi_version -- PKV_ABI_VERSION of the loaded library. */
+int pkv_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

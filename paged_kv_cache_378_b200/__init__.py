@@ -1,0 +1,194 @@
+"""Paged KV-cache decode path for B200 (sm_100a): thin Python binding.
+
+Every function here only checks and marshals arguments (torch CUDA tensors
+-> raw device pointers + sizes + the current CUDA stream) and calls the C ABI
+of ``libpagedkv.so`` (``include/pagedkv.h``); all work runs in the library's
+CUDA kernels.  There is no CPU path: without the library, calls raise.
+
+Names follow the pages' statement of the problem:
+
+* ``kv_append(k, v, slot_mapping, k_pool, v_pool)`` -- new tokens fill their
+  slots ("Infra: PagedAttention", section 按 Block 分配).
+* ``paged_decode_attention(q, k_pool, v_pool, block_tables, seq_lens,
+  block_size, scale, out)`` -- attention read through block tables, split
+  into partitions merged by the max-rescaled rule (same section).
+* ``block_copy(src_dst_pairs, k_pool, v_pool)`` -- copy-on-write of shared
+  tail blocks (section 共享前缀，分叉时 Copy-on-write).
+
+Pool tensors are bf16 ``[num_layers, num_blocks, num_kv_heads, block_size,
+head_dim]`` (or without the leading layer dimension for one layer).
+"""
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import PkvCache
+
+__all__ = [
+    "PagedKVError", "kv_append", "block_copy", "paged_decode_attention",
+    "attention_workspace_bytes", "partition_tokens", "make_workspace",
+    "get_device_status", "library", "DEV_RANGE", "DEV_LENGTH", "DEV_TIMEOUT",
+]
+
+DEV_RANGE = 0x1
+DEV_LENGTH = 0x2
+DEV_TIMEOUT = 0x4
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        msg = library().pkv_strerror(code).decode()
+        super().__init__(f"{where}: {msg} (status {code})")
+
+
+def library():
+    return _lib.load()
+
+
+def _check(rc, where):
+    if rc != 0:
+        raise PagedKVError(rc, where)
+
+
+def _need(t, name, dtype, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _pool_dims(k_pool, v_pool):
+    _need(k_pool, "k_pool", torch.bfloat16)
+    _need(v_pool, "v_pool", torch.bfloat16, k_pool.device)
+    if k_pool.shape != v_pool.shape:
+        raise ValueError("k_pool and v_pool shapes differ")
+    if k_pool.dim() == 4:
+        L = 1
+        NB, H, B, D = k_pool.shape
+    elif k_pool.dim() == 5:
+        L, NB, H, B, D = k_pool.shape
+    else:
+        raise ValueError("pools must be [L, NB, H_kv, B, d] or [NB, H_kv, B, d]")
+    return L, NB, H, B, D
+
+
+def _cache(k_pool, v_pool):
+    L, NB, H, B, D = _pool_dims(k_pool, v_pool)
+    c = PkvCache(k_pool.data_ptr(), v_pool.data_ptr(), L, NB, H, B, D)
+    return c, (L, NB, H, B, D)
+
+
+def _stream(device, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def kv_append(k, v, slot_mapping, k_pool, v_pool, layer=0, stream=None):
+    """Store new tokens' K/V (bf16 ``[T, H_kv, d]``) at ``slot_mapping`` (int64 ``[T]``).
+
+    ``slot < 0`` skips the token (padding).  Bit-exact copy.
+    """
+    cache, (L, NB, H, B, D) = _cache(k_pool, v_pool)
+    dev = k_pool.device
+    _need(k, "k", torch.bfloat16, dev)
+    _need(v, "v", torch.bfloat16, dev)
+    _need(slot_mapping, "slot_mapping", torch.int64, dev)
+    T = slot_mapping.numel()
+    if k.shape != (T, H, D) or v.shape != (T, H, D):
+        raise ValueError(f"k/v must be [{T}, {H}, {D}]")
+    rc = library().pkv_kv_append(ctypes.byref(cache), int(layer), k.data_ptr(), v.data_ptr(),
+                                 slot_mapping.data_ptr(), T, _stream(dev, stream))
+    _check(rc, "kv_append")
+
+
+def block_copy(src_dst_pairs, k_pool, v_pool, stream=None):
+    """Copy whole blocks (every layer, K and V): ``pool[:, dst] = pool[:, src]``.
+
+    ``src_dst_pairs``: int32 ``[n, 2]``.
+    """
+    cache, _ = _cache(k_pool, v_pool)
+    dev = k_pool.device
+    _need(src_dst_pairs, "src_dst_pairs", torch.int32, dev)
+    if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be [n, 2]")
+    n = src_dst_pairs.shape[0]
+    rc = library().pkv_block_copy(ctypes.byref(cache), src_dst_pairs.data_ptr(), n,
+                                  _stream(dev, stream))
+    _check(rc, "block_copy")
+
+
+def attention_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                              block_size, partition_tokens=0):
+    return int(library().pkv_attention_workspace_bytes(
+        num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, block_size,
+        partition_tokens))
+
+
+def partition_tokens(num_seqs, num_kv_heads, head_dim, max_blocks_per_seq, block_size, requested=0):
+    """Partition length the attention call will use (0 = library default)."""
+    return int(library().pkv_partition_tokens(num_seqs, num_kv_heads, head_dim, max_blocks_per_seq,
+                                              block_size, requested))
+
+
+def make_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, block_size,
+                   partition_tokens=0, device="cuda"):
+    """A zeroed workspace for these sizes (zeroed once; the kernel keeps it ready)."""
+    n = attention_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                  max_blocks_per_seq, block_size, partition_tokens)
+    if n == 0:
+        raise ValueError("invalid sizes for the attention workspace")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def paged_decode_attention(q, k_pool, v_pool, block_tables, seq_lens, block_size, scale, out,
+                           layer=0, workspace=None, partition_tokens=0, stream=None):
+    """Decode attention through block tables; writes bf16 ``out [N, H_q, d]``.
+
+    ``q`` bf16 ``[N, H_q, d]``; ``block_tables`` int32 ``[N, max_blocks]``;
+    ``seq_lens`` int32 ``[N]``; ``scale`` usually ``1/sqrt(d)``.
+    ``workspace``: uint8 CUDA tensor from ``make_workspace`` (required when a
+    sequence can span several partitions).
+    """
+    cache, (L, NB, H, B, D) = _cache(k_pool, v_pool)
+    if int(block_size) != B:
+        raise ValueError(f"block_size {block_size} does not match the pools ({B})")
+    dev = k_pool.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(out, "out", torch.bfloat16, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    if q.dim() != 3 or q.shape[2] != D:
+        raise ValueError(f"q must be [N, H_q, {D}]")
+    N, Hq, _ = q.shape
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    if block_tables.dim() != 2 or block_tables.shape[0] != N or seq_lens.shape != (N,):
+        raise ValueError("block_tables must be [N, max_blocks] and seq_lens [N]")
+    maxb = block_tables.shape[1]
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8, dev)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+    rc = library().pkv_paged_decode_attention(
+        ctypes.byref(cache), int(layer), q.data_ptr(), N, Hq, block_tables.data_ptr(), maxb,
+        seq_lens.data_ptr(), float(scale), out.data_ptr(), ws_ptr, ws_bytes, int(partition_tokens),
+        _stream(dev, stream))
+    _check(rc, "paged_decode_attention")
+    return out
+
+
+def get_device_status(reset=True):
+    """Device status bits (DEV_RANGE | DEV_LENGTH | DEV_TIMEOUT); synchronises the device."""
+    v = ctypes.c_uint(0)
+    _check(library().pkv_get_device_status(ctypes.byref(v), 1 if reset else 0), "get_device_status")
+    return int(v.value)

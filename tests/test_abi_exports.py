@@ -1,0 +1,105 @@
+"""The C ABI library builds, loads and exports every symbol include/pagedkv.h
+declares; its host-side argument checks answer before any launch (no GPU
+needed: every call here returns before touching the device)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+
+import paged_kv_cache_378_b200 as pkv
+from paged_kv_cache_378_b200 import _lib
+from paged_kv_cache_378_b200.build import INCLUDE
+
+HEADER = os.path.join(INCLUDE, "pagedkv.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert _declared() == sorted(_lib.SIGNATURES)
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = pkv.library()
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.lib_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (pkv_[a-z_]+)$", out, flags=re.M))
+    assert set(_declared()) <= exported
+
+
+def test_version_and_error_strings():
+    lib = pkv.library()
+    assert lib.pkv_abi_version() == 1
+    for code in range(0, -8, -1):
+        assert lib.pkv_strerror(code)
+    assert b"unknown" in lib.pkv_strerror(-99)
+
+
+def _cache(**kw):
+    d = dict(k_pool=16, v_pool=32, num_layers=1, num_blocks=8, num_kv_heads=2, block_size=16,
+             head_dim=64)
+    d.update(kw)
+    return _lib.PkvCache(d["k_pool"], d["v_pool"], d["num_layers"], d["num_blocks"],
+                         d["num_kv_heads"], d["block_size"], d["head_dim"])
+
+
+def test_host_argument_checks_before_launch():
+    lib = pkv.library()
+    P = ctypes.byref
+    c = _cache()
+    # NULL cache / pools
+    assert lib.pkv_kv_append(None, 0, 16, 16, 16, 1, None) == -1
+    assert lib.pkv_block_copy(P(_cache(k_pool=0)), 16, 1, None) == -1
+    # unsupported shapes
+    assert lib.pkv_kv_append(P(_cache(head_dim=96)), 0, 16, 16, 16, 1, None) == -5
+    assert lib.pkv_kv_append(P(_cache(block_size=4)), 0, 16, 16, 16, 1, None) == -5
+    assert lib.pkv_kv_append(P(_cache(num_blocks=0)), 0, 16, 16, 16, 1, None) == -2
+    # misaligned pool / inputs
+    assert lib.pkv_kv_append(P(_cache(k_pool=18)), 0, 16, 16, 16, 1, None) == -3
+    assert lib.pkv_kv_append(P(c), 0, 24, 16, 16, 1, None) == -3
+    # layer range, negative counts, empty work (returns before any launch)
+    assert lib.pkv_kv_append(P(c), 1, 16, 16, 16, 1, None) == -7
+    assert lib.pkv_kv_append(P(c), 0, 16, 16, 16, -1, None) == -2
+    assert lib.pkv_kv_append(P(c), 0, None, None, None, 0, None) == 0
+    assert lib.pkv_block_copy(P(c), None, 0, None) == 0
+    assert lib.pkv_block_copy(P(c), None, 3, None) == -1
+    assert lib.pkv_block_copy(P(c), 16, -2, None) == -2
+    att = lib.pkv_paged_decode_attention
+    # H_q not a multiple of H_kv, unsupported group, bad scale
+    assert att(P(c), 0, 16, 2, 3, 16, 4, 16, 0.125, 16, None, 0, 0, None) == -2
+    assert att(P(c), 0, 16, 2, 6, 16, 4, 16, 0.125, 16, None, 0, 0, None) == -5
+    assert att(P(c), 0, 16, 2, 8, 16, 4, 16, float("nan"), 16, None, 0, 0, None) == -2
+    assert att(P(c), 0, 16, 0, 8, 16, 4, 16, 0.125, 16, None, 0, 0, None) == 0
+    assert att(P(c), 0, None, 2, 8, 16, 4, 16, 0.125, 16, None, 0, 0, None) == -1
+    assert att(P(c), 0, 16, 2, 8, 16, 4, 16, 0.125, 40, None, 0, 0, None) == -3
+    # a table that spans several partitions needs a workspace of the right size
+    assert att(P(c), 0, 16, 2, 8, 16, 4096, 16, 0.125, 16, None, 0, 512, None) == -4
+    need = lib.pkv_attention_workspace_bytes(2, 8, 2, 64, 4096, 16, 512)
+    assert need > 0
+    assert att(P(c), 0, 16, 2, 8, 16, 4096, 16, 0.125, 16, 256, need - 1, 512, None) == -4
+
+
+def test_workspace_and_partition_sizes():
+    lib = pkv.library()
+    # partition rounds up to the tile (16 tokens, or the block when larger)
+    assert lib.pkv_partition_tokens(8, 8, 128, 2048, 16, 500) == 512
+    assert lib.pkv_partition_tokens(8, 8, 128, 2048, 32, 40) == 64
+    assert lib.pkv_partition_tokens(8, 8, 64, 2048, 8, 1) == 16
+    assert lib.pkv_partition_tokens(8, 8, 96, 2048, 8, 1) == -1
+    d = lib.pkv_partition_tokens(64, 8, 64, 128, 16, 0)
+    assert d >= 256 and d % 16 == 0
+    # bytes grow with the number of partitions: (G*d + G*2) floats per partition + counters
+    n1 = lib.pkv_attention_workspace_bytes(8, 32, 8, 128, 2048, 16, 512)
+    parts = 32768 // 512
+    units = 8 * 8
+    assert n1 >= units * parts * 4 * (128 + 2) * 4 + units * 4
+    assert lib.pkv_attention_workspace_bytes(8, 30, 8, 128, 2048, 16, 512) == 0
+    assert lib.pkv_attention_workspace_bytes(8, 32, 8, 128, 2048, 12, 512) == 0
