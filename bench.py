@@ -90,7 +90,7 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, pci_bus_id=None, period_ms=100):
-        self.pci = (pci_bus_id or "").lower()
+        self.pci = (pci_bus_id or "").strip().lower()
         self.period_ms = period_ms
         self.rows = []
         self.proc = None
@@ -100,7 +100,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 f"-lms={self.period_ms}"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                 "-lms", str(self.period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                 text=True)
         except OSError:
             self.proc = None
@@ -153,10 +153,25 @@ def pci_bus_id(dev):
         from cuda.bindings import runtime as rt
         err, bus = rt.cudaDeviceGetPCIBusId(32, dev)
         if int(err) == 0:
-            return bus.decode().rstrip("\x00") if isinstance(bus, bytes) else str(bus)
+            bus = bus.decode() if isinstance(bus, bytes) else str(bus)
+            return bus.replace("\x00", "").strip()
     except Exception:
         pass
     return None
+
+
+def combine_over_ranks(dist, ms, nbytes, nseqs, device):
+    """(max device ms, total bytes, total sequences) over all ranks.
+
+    Every rank must call this the same number of times, in the same order.
+    """
+    if dist is None:
+        return float(ms), float(nbytes), float(nseqs)
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    w = torch.tensor([nbytes, nseqs], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return float(t[0]), float(w[0]), float(w[1])
 
 
 # ---------------------------------------------------------------------------
@@ -392,7 +407,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
-    ap.add_argument("--soak-seconds", type=float, default=1.0)
+    ap.add_argument("--soak-seconds", type=float, default=1.5)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -420,6 +435,8 @@ def main():
     part = spec.partition_tokens if args.partition < 0 else args.partition
     seed = rank_seed(spec.seed, rank)
 
+    sampler = ClockSampler(pci_bus_id(local)).start()   # warms up while the inputs are built
+
     # cpu baseline first, before the GPU is busy (rank 0 at N = 1 only)
     w_meta = make_workload(args.workload, block_size=B, seed=seed, values=False)
     unique_bytes = w_meta.unique_kv_bytes_read()
@@ -443,8 +460,6 @@ def main():
     if pkv.get_device_status(reset=True):
         raise SystemExit("device status raised during warm-up")
 
-    sampler = ClockSampler(pci_bus_id(local)).start()
-    time.sleep(0.3)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps * spec.num_layers)]
     t_start = torch.cuda.Event(enable_timing=True)
@@ -482,26 +497,16 @@ def main():
     attn_ms = [a.elapsed_time(b) for a, b in evs]
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
 
-    # totals over ranks
-    ms_max = ms
-    bytes_total = unique_bytes * spec.num_layers
-    seqs_total = w.num_seqs
-    if dist is not None:
-        t = torch.tensor([ms, bytes_total, seqs_total], dtype=torch.float64, device=device)
-        tm = t.clone()
-        dist.all_reduce(tm[0:1], op=dist.ReduceOp.MAX)
-        dist.all_reduce(tm[1:3], op=dist.ReduceOp.SUM)
-        ms_max, bytes_total, seqs_total = float(tm[0]), float(tm[1]), float(tm[2])
+    # totals over ranks: device time is the max, work is the sum
+    ms_max, bytes_total, seqs_total = combine_over_ranks(
+        dist, ms, unique_bytes * spec.num_layers, w.num_seqs, device)
     ms_per_step = ms_max / args.steps
     value = bytes_total / (ms_per_step * 1e-3) / 1e9
 
     e2e = None
     if not args.no_e2e:
         e_ms, h2d, d2h = e2e_run(pkv, w, gs, args.e2e_steps, device)
-        if dist is not None:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t[0])
+        e_ms = combine_over_ranks(dist, e_ms, 0, 0, device)[0]
         e2e = {"value": bytes_total / (e_ms * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e_ms, "steps": args.e2e_steps}

@@ -38,7 +38,7 @@
  * s % block_size of physical block s / block_size, as in the page's example:
  * with table [3, 0, 4] and B = 4, position 8 is logical block 2 -> P4, row 0.
  *
- * Supported shapes: head_dim in {64, 128}; block_size in {8, 16, 32};
+ * Supported shapes: head_dim in {64, 128}; block_size in {4, 8, 16, 32};
  * num_q_heads = G * num_kv_heads with G in {1, 2, 4, 8}.  Query head h
  * reads kv head h / G (contiguous GQA groups).
  */
@@ -120,19 +120,21 @@ int pkv_block_copy(const pkv_cache_t* cache, const int32_t* src_dst_pairs,
 
 /*
  * pkv_attention_workspace_bytes -- bytes of workspace pkv_paged_decode_attention
- * needs for these sizes (split-K partials plus one counter per (sequence,
- * kv head)).  `partition_tokens` as passed to the attention call (0 = the
- * library's choice).  Returns 0 for invalid sizes.
+ * needs for these sizes on the current device: the work plan (a prefix of
+ * tiles per sequence and the start of every work range), the partial results
+ * of sequences split across ranges, and one ticket per (sequence, kv head).
+ * `partition_tokens` as passed to the attention call.  Returns 0 for invalid
+ * sizes.
  */
 size_t pkv_attention_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,
                                      int head_dim, int max_blocks_per_seq, int block_size,
                                      int partition_tokens);
 
 /*
- * pkv_partition_tokens -- the KV partition length (tokens) the attention call
- * uses for these sizes; `requested` 0 picks the library's default, otherwise
- * it is rounded up to the kernel's tile (16 tokens, or the block size when
- * larger).  Returns <= 0 for invalid sizes.
+ * pkv_partition_tokens -- the longest work range (tokens) the attention call
+ * uses: `requested` rounded up to the kernel's tile (32 tokens at head_dim 64,
+ * 16 at head_dim 128 or with 4-token blocks, never less than one block), or 0
+ * when `requested` is 0 (no cap).  Returns < 0 for invalid sizes.
  */
 int pkv_partition_tokens(int num_seqs, int num_kv_heads, int head_dim,
                          int max_blocks_per_seq, int block_size, int requested);
@@ -152,12 +154,14 @@ int pkv_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
  * the block table and reads the physical blocks in place, without copying
  * them into one contiguous range (ithelp article 10405755, "PagedAttention
  * 的核心想法"; "Infra: PagedAttention", "按 Block 分配").  Score
- * s_i = scale * q . k_i, softmax over every visible token.  Long sequences
- * are split into partitions of `partition_tokens` tokens; each partition
- * keeps (max score m_r, Z_r = sum e^{s_i - m_r}, unnormalised output) and the
- * partitions are merged with o = sum_r e^{m_r - M} Z_r o_r / sum_r e^{m_r - M} Z_r,
+ * s_i = scale * q . k_i, softmax over every visible token.  The work over all
+ * (sequence, kv head) pairs is cut into one range per warp plus small ranges
+ * claimed dynamically; a sequence that spans several ranges is computed in
+ * pieces, each keeping (max score
+ * m_r, Z_r = sum e^{s_i - m_r}, unnormalised output), and the pieces are
+ * merged with o = sum_r e^{m_r - M} Z_r o_r / sum_r e^{m_r - M} Z_r,
  * M = max_r m_r ("Infra: PagedAttention", "按 Block 分配", the merge
- * equation and the paragraph on max rescaling).
+ * equation and the paragraph on max rescaling).  One kernel launch.
  *
  *   layer              layer of the pools to read
  *   q                  bf16 [num_seqs][num_q_heads][head_dim]
@@ -172,11 +176,13 @@ int pkv_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
  *   out                bf16 [num_seqs][num_q_heads][head_dim], round to
  *                      nearest even from fp32
  *   workspace          device buffer of at least
- *                      pkv_attention_workspace_bytes(...) bytes, 16-byte
- *                      aligned, zeroed once (pkv_workspace_init) before its
- *                      first use; may be NULL only if every sequence fits in
- *                      one partition (max_blocks_per_seq*B <= partition)
- *   partition_tokens   0 = library default, else the split-K partition length
+ *                      pkv_attention_workspace_bytes(...) bytes (same sizes,
+ *                      same device), 16-byte aligned, zeroed once
+ *                      (pkv_workspace_init) before its first use; the call
+ *                      leaves it ready for the next call.  After a launch
+ *                      that raised PKV_DEV_TIMEOUT, zero it again.
+ *   partition_tokens   0 = no cap on the ranges; > 0 = no range longer than
+ *                      this many tokens (rounded up to the tile)
  * Concurrent calls must not share a workspace.
  */
 int pkv_paged_decode_attention(const pkv_cache_t* cache, int layer,

@@ -1,0 +1,540 @@
+// Paged decode attention: one persistent grid, work split evenly per warp.
+//
+// What is computed ("Infra: PagedAttention", section 按 Block 分配; ithelp
+// article 10405755, section PagedAttention 的核心想法): per (sequence, kv
+// head) and each of its G query heads, softmax(scale * q . k_i) over all the
+// sequence's tokens, read in place through the block table, times V.  Work
+// computed in pieces is merged with the page's max-rescaled rule
+//     o = sum_r e^{m_r - M} o_r / sum_r e^{m_r - M} Z_r,   M = max_r m_r.
+//
+// Decomposition.  Every (sequence, kv head) is a unit of ceil(len/TILE)
+// tiles; units are laid end to end (sequence-major, kv head minor) into one
+// flat space of T tiles, cut into R ranges of equal length.  Without a
+// partition cap R is the number of warps in the grid (one range each); with
+// a cap of C tiles, each warp takes ceil(ceil(T/C)/K) consecutive ranges.
+// A warp streams its tiles with one continuous bulk-copy pipeline that runs
+// across unit and range boundaries, so it never drains between sequences,
+// and every warp gets the same number of tiles whatever the length mix.  A
+// unit inside one range is finished by its warp; a unit cut by range
+// boundaries leaves one partial per range, and the last range to finish (an
+// atomic ticket per unit, reset by that range) merges them in range order,
+// so the result does not depend on which piece finishes last.
+//
+// Planning.  Every CTA reads the sequence lengths once and scans them into
+// a prefix of tiles per sequence, kept in shared memory (in global memory,
+// written identically by every CTA, for batches of more than PREFIX_SMEM
+// sequences); a warp finds its first tile by binary search.
+//
+// Data movement.  Each warp owns a ring of STAGES shared-memory stages.  One
+// lane issues, per stage, TMA tensor loads (cp.async.bulk.tensor, 2-D tensor
+// map over all pool rows, 128-byte swizzle, no multicast) of the tile's
+// physical blocks for K and V, plus a bulk copy of the unit's q when the unit
+// starts; all complete on the stage's mbarrier.  The swizzle makes the
+// ldmatrix reads of K and V conflict-free.  Rows of a tail block past the
+// sequence's length are loaded with the block but masked: their scores are
+// -inf and their V rows are zeroed in shared memory before the P V product.
+//
+// Compute.  Tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with
+// the G query heads as the MMA rows; see attn_common.cuh.
+//
+// Faults never trap: waits are bounded (a timeout sets PKV_DEV_TIMEOUT,
+// drains this warp's copies in flight and returns), block ids outside the
+// pool set PKV_DEV_RANGE and are not fetched, lengths above the table's
+// capacity set PKV_DEV_LENGTH and are clamped.
+#pragma once
+
+#include <cuda.h>
+
+#include "attn_common.cuh"
+
+namespace pkv {
+
+struct AttnArgs {
+    const uint16_t* q;             // [N][Hq][D]
+    uint16_t* out;                 // [N][Hq][D]
+    const int32_t* block_tables;   // [N][max_blocks]
+    const int32_t* seq_lens;       // [N]
+    int num_seqs;
+    int num_kv_heads;
+    int num_blocks;
+    int max_blocks;
+    float qscale;                  // scale * log2(e)
+    long long row_base;            // pool row of (layer, block 0, head 0, row 0) in the tensor maps
+    // workspace
+    float2* part_mz;               // [R_max][2][G]    (m, Z) of a partial, base 2
+    float* part_o;                 // [R_max][2][G][D] unnormalised partial output
+    unsigned int* tickets;         // [N*Hkv] zero at rest
+    long long* prefix_g;           // [N+1] tile prefix, used when N > PREFIX_SMEM
+    int R_max;                     // ranges the workspace holds
+    int cap_tiles;                 // > 0: no range longer than this many tiles
+    int K;                         // warps in the grid
+};
+
+constexpr int PREFIX_SMEM = 1024;      // sequences whose tile prefix fits in shared memory
+
+// R equal ranges over the flat space of T tiles (R <= T, so none is empty).
+struct Sched {
+    long long T, R;
+    __device__ __forceinline__ long long begin(long long r) const { return r * T / R; }
+    // the range holding flat tile t: the largest r with begin(r) <= t
+    __device__ __forceinline__ long long range_of(long long t) const { return ((t + 1) * R - 1) / T; }
+};
+
+__device__ __forceinline__ int clamp_len(int len, int cap) { return len > cap ? cap : (len < 0 ? 0 : len); }
+
+template <int D, int G, int BS, int NW, int STAGES>
+struct AttnCfg {
+    using TS = TileSmem<D, BS>;
+    static constexpr int TILE = TS::TILE;
+    static constexpr int BPT = TS::BPT;
+    static constexpr int KT_BYTES = TS::KT_BYTES;
+    static constexpr int STAGE_BYTES = 2 * KT_BYTES;            // K tile, V tile
+    static constexpr int Q_BYTES = G * D * 2;                   // q of a unit
+    static constexpr int META_BYTES = 32;
+    static constexpr int RING_BYTES = NW * STAGES * STAGE_BYTES;
+    static constexpr int Q_OFF = RING_BYTES;
+    static constexpr int META_OFF = Q_OFF + NW * STAGES * Q_BYTES;
+    static constexpr int BAR_OFF = META_OFF + NW * STAGES * META_BYTES;
+    static constexpr int PREFIX_OFF = BAR_OFF + NW * STAGES * 8;
+    static constexpr int SMEM_BYTES = PREFIX_OFF + (PREFIX_SMEM + 1) * 4 + 1024;   // + alignment slack
+    static constexpr int BOX_BYTES = BS * 128;                  // one TMA box: BS rows x 64 dims
+    static constexpr int NT = NW * 32;
+};
+
+struct StageMeta {
+    int s, h, t, len;
+    long long f;      // flat tile index
+    int flags;
+    int r;            // range
+};
+static_assert(sizeof(StageMeta) == 32, "meta layout");
+
+constexpr int F_FIRST = 1;        // first tile of a unit within this range: q staged, state reset
+constexpr int F_LAST = 2;         // last tile of a unit within this range: finish the unit
+constexpr int F_UNIT_START = 4;   // tile 0 of the unit
+constexpr int F_UNIT_END = 8;     // last tile of the unit
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Block-wide exclusive scan of one value per thread (NT threads); returns
+// the thread's exclusive prefix and writes the block total to *total.
+template <int NT>
+__device__ __forceinline__ long long block_scan(long long v, long long* s_red, long long* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    long long x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const long long y = __shfl_up_sync(FULL, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) s_red[warp] = x;
+    __syncthreads();
+    long long before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
+        const long long sw = s_red[w];
+        if (w < warp) before += sw;
+        all += sw;
+    }
+    __syncthreads();
+    *total = all;
+    return before + x - v;
+}
+
+// register budgets: at least this many warps resident per SM (head_dim 64 / 128)
+#ifndef PKV_ATTN_MIN_WARPS_PER_SM
+#define PKV_ATTN_MIN_WARPS_PER_SM 12
+#endif
+#ifndef PKV_ATTN_MIN_WARPS_PER_SM_128
+#define PKV_ATTN_MIN_WARPS_PER_SM_128 8
+#endif
+
+template <int D, int G, int BS, int NW, int STAGES>
+__global__ void __launch_bounds__(NW * 32, (D == 64 ? PKV_ATTN_MIN_WARPS_PER_SM : PKV_ATTN_MIN_WARPS_PER_SM_128) / NW)
+paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                       const __grid_constant__ CUtensorMap tmap_v, const AttnArgs a) {
+    using C = AttnCfg<D, G, BS, NW, STAGES>;
+    using TS = typename C::TS;
+    constexpr int TILE = C::TILE;
+    constexpr int NT = C::NT;
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ long long s_red[NW];
+
+    // 1024-byte aligned base (swizzled TMA destinations)
+    const uint32_t raw_addr = smem_addr(smem_raw);
+    unsigned char* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int tid = threadIdx.x;
+    unsigned char* ring = smem + (size_t)warp * STAGES * C::STAGE_BYTES;
+    unsigned char* qslots = smem + C::Q_OFF + (size_t)warp * STAGES * C::Q_BYTES;
+    StageMeta* meta = reinterpret_cast<StageMeta*>(smem + C::META_OFF) + warp * STAGES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF) + warp * STAGES;
+
+    if (lane == 0) {
+        if (warp == 0) {
+            prefetch_tensormap(&tmap_k);
+            prefetch_tensormap(&tmap_v);
+        }
+#pragma unroll
+        for (int st = 0; st < STAGES; ++st) mbar_init(smem_addr(&bars[st]), 1);
+        fence_mbar_init();
+    }
+
+    const int N = a.num_seqs;
+    const int Hkv = a.num_kv_heads;
+    const int Hq = Hkv * G;
+    const int cap = a.max_blocks * BS;
+    const bool pre_smem = N <= PREFIX_SMEM;
+    int* s_prefix = reinterpret_cast<int*>(smem + C::PREFIX_OFF);
+
+    // ---- plan: prefix of tiles per sequence, T, the schedule -------------------------
+    long long T = 0;
+    for (int base = 0; base < N; base += NT) {
+        const int s = base + tid;
+        long long v = 0;
+        if (s < N) {
+            const int raw = __ldg(a.seq_lens + s);
+            const int len = clamp_len(raw, cap);
+            v = (long long)Hkv * ((len + TILE - 1) / TILE);
+            if (blockIdx.x == 0) {
+                if (raw > cap) raise_status(PKV_DEV_LENGTH);
+                if (len == 0) {   // nothing to attend to: zero output
+                    uint4* o4 = reinterpret_cast<uint4*>(a.out + (size_t)s * Hq * D);
+                    for (int c = 0; c < Hq * D / 8; ++c) o4[c] = make_uint4(0, 0, 0, 0);
+                }
+            }
+        }
+        long long tot;
+        const long long incl = T + block_scan<NT>(v, s_red, &tot) + v;
+        if (s < N) {
+            if (pre_smem) s_prefix[s + 1] = (int)incl;
+            else a.prefix_g[s + 1] = incl;     // every CTA writes the same values
+        }
+        T += tot;
+    }
+    if (tid == 0) {
+        if (pre_smem) s_prefix[0] = 0;
+        else a.prefix_g[0] = 0;
+    }
+    const long long K = a.K;
+    Sched sc;
+    sc.T = T;
+    long long rpw = 1;                                    // ranges per warp
+    if (a.cap_tiles > 0 && T > 0) {
+        const long long need = (T + a.cap_tiles - 1) / a.cap_tiles;
+        rpw = (need + K - 1) / K;
+    }
+    sc.R = K * rpw;
+    if (sc.R > T) sc.R = T;
+    if (sc.R > a.R_max) {                                 // cannot happen with a workspace of the queried size
+        if (tid == 0 && blockIdx.x == 0) raise_status(PKV_DEV_RANGE);
+        sc.R = a.R_max;
+    }
+    __syncthreads();
+    const long long wg = (long long)blockIdx.x * NW + warp;
+    const long long r_first = wg * rpw;
+    const long long r_stop = r_first + rpw < sc.R ? r_first + rpw : sc.R;   // this warp's ranges
+
+    // (sequence, kv head, tile) of flat tile f: largest s with prefix[s] <= f
+    auto locate = [&](long long f, int& s_out, int& h_out, int& t_out) {
+        int lo = 0, hi = N - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            const long long pm = pre_smem ? (long long)s_prefix[mid] : a.prefix_g[mid];
+            if (pm <= f) lo = mid; else hi = mid - 1;
+        }
+        const long long p0 = pre_smem ? (long long)s_prefix[lo] : a.prefix_g[lo];
+        const long long p1 = pre_smem ? (long long)s_prefix[lo + 1] : a.prefix_g[lo + 1];
+        const long long nt = (p1 - p0) / Hkv;
+        const long long off = f - p0;
+        s_out = lo;
+        h_out = (int)(off / nt);
+        t_out = (int)(off % nt);
+    };
+
+    const uint64_t pol_stream = policy_evict_first();
+
+    // ---- producer cursor (every lane keeps an identical copy) ------------------
+    long long r = r_first;                                // range of the next tile to issue
+    long long f = 0, f_end = 0, f_stop = 0;
+    int ps = 0, ph = 0, pt = 0, plen = 0, pnt = 0, next_len = 0;
+    bool range_first = true;
+    int ids = -1, ids_seq = -1, ids_base = 0;
+    int pre = -1, pre_seq = -1, pre_base = 0;
+
+    auto load_batch = [&](int s, int base, int len) -> int {
+        const int lb = base + lane;
+        return (lb * BS < len) ? __ldg(a.block_tables + (size_t)s * a.max_blocks + lb) : -1;
+    };
+    auto seq_len = [&](int s) -> int { return s < N ? clamp_len(__ldg(a.seq_lens + s), cap) : 0; };
+    auto advance_unit = [&]() {
+        pt = 0;
+        if (++ph < Hkv) return;
+        ph = 0;
+        ++ps;
+        plen = next_len;
+        pnt = (plen + TILE - 1) / TILE;
+        while (pnt == 0 && ps + 1 < N) {   // skip empty sequences (rare, synchronous)
+            ++ps;
+            plen = seq_len(ps);
+            pnt = (plen + TILE - 1) / TILE;
+        }
+        next_len = seq_len(ps + 1);
+    };
+    const bool have_work = r_first < r_stop;
+    if (have_work) {
+        f = sc.begin(r_first);
+        f_end = sc.begin(r_first + 1);
+        f_stop = sc.begin(r_stop);
+        locate(f, ps, ph, pt);
+        plen = seq_len(ps);
+        pnt = (plen + TILE - 1) / TILE;
+        next_len = seq_len(ps + 1);
+    }
+
+    // Stage the next tile into stage `st`; false when this warp has no more tiles.
+    auto issue = [&](int st) -> bool {
+        if (f == f_stop) return false;
+        if (f == f_end) {                                 // next range of this warp (contiguous)
+            ++r;
+            f_end = sc.begin(r + 1);
+            range_first = true;
+        }
+        const int nv = min(TILE, plen - pt * TILE);
+        int flags = 0;
+        if (pt == 0) flags |= F_UNIT_START;
+        if (pt == pnt - 1) flags |= F_UNIT_END;
+        if (range_first || pt == 0) flags |= F_FIRST;
+        if (f + 1 == f_end || pt == pnt - 1) flags |= F_LAST;
+        range_first = false;
+        const int lb0 = pt * C::BPT;
+        if (ids_seq != ps || lb0 < ids_base || lb0 + C::BPT > ids_base + 32) {
+            if (pre_seq == ps && lb0 >= pre_base && lb0 + C::BPT <= pre_base + 32) {
+                ids = pre; ids_seq = pre_seq; ids_base = pre_base;
+            } else {
+                ids = load_batch(ps, lb0, plen); ids_seq = ps; ids_base = lb0;
+            }
+            // prefetch the batch needed after this one: the rest of this table
+            // row, else the row's start again for the next kv head, else the
+            // next sequence's row
+            if ((ids_base + 32) * BS < plen) {
+                pre_seq = ps; pre_base = ids_base + 32; pre = load_batch(ps, pre_base, plen);
+            } else if (ph + 1 < Hkv && ids_base != 0) {
+                pre_seq = ps; pre_base = 0; pre = load_batch(ps, 0, plen);
+            } else if (ps + 1 < N) {
+                pre_seq = ps + 1; pre_base = 0; pre = load_batch(ps + 1, 0, next_len);
+            }
+        }
+        int bid[C::BPT];
+#pragma unroll
+        for (int j = 0; j < C::BPT; ++j) bid[j] = __shfl_sync(FULL, ids, lb0 - ids_base + j);
+        if (lane == 0) {
+            StageMeta m;
+            m.s = ps; m.h = ph; m.t = pt; m.len = plen; m.f = f; m.flags = flags; m.r = (int)r;
+            meta[st] = m;
+            const uint32_t bar = smem_addr(&bars[st]);
+            const uint32_t dK = smem_addr(ring + (size_t)st * C::STAGE_BYTES);
+            const uint32_t dV = dK + C::KT_BYTES;
+            uint32_t bytes = (flags & F_FIRST) ? C::Q_BYTES : 0u;
+            bool bad = false;
+#pragma unroll
+            for (int j = 0; j < C::BPT; ++j) {
+                if (j * BS >= nv) continue;
+                if (bid[j] < 0 || bid[j] >= a.num_blocks) { bad = true; continue; }
+                bytes += 2u * TS::HALVES * C::BOX_BYTES;
+            }
+            if (bad) raise_status(PKV_DEV_RANGE);
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(bar, bytes);
+            if (flags & F_FIRST)
+                bulk_g2s(smem_addr(qslots + (size_t)st * C::Q_BYTES),
+                         a.q + ((size_t)ps * Hq + (size_t)ph * G) * D, C::Q_BYTES, bar, pol_stream);
+#pragma unroll
+            for (int j = 0; j < C::BPT; ++j) {
+                if (j * BS >= nv || bid[j] < 0 || bid[j] >= a.num_blocks) continue;
+                // pool row of (layer, block, head, row 0); the layer is in row_base
+                const int y = (int)(a.row_base + ((long long)bid[j] * Hkv + ph) * BS);
+                const uint32_t off = (uint32_t)(j * TS::RPB * 128);
+#pragma unroll
+                for (int hf = 0; hf < TS::HALVES; ++hf) {
+                    tma_load_2d(dK + hf * TS::HALF_BYTES + off, &tmap_k, 64 * hf, y, bar, pol_stream);
+                    tma_load_2d(dV + hf * TS::HALF_BYTES + off, &tmap_v, 64 * hf, y, bar, pol_stream);
+                }
+            }
+        }
+        ++f;
+        if (++pt == pnt) advance_unit();
+        return true;
+    };
+
+    // ---- finishing a unit --------------------------------------------------------
+    MmaState<D> ws;
+    ws.reset();
+    uint32_t qa[D / 16][4];
+    bool began = false;
+    const int g_row = lane >> 2;    // query head of this lane's fragment row
+    const int c4 = lane & 3;
+
+    // Finish this warp's share of unit (m.s, m.h).  A unit computed entirely
+    // here is normalised and written.  A piece of a split unit is stored as a
+    // partial of its range; the piece that completes the unit's ticket merges
+    // every partial of the unit in range order (max rescaled) and writes bf16.
+    auto finish_unit = [&](const StageMeta& m) {
+        // full row sums: the 4 lanes of a row own disjoint columns
+        float l = ws.l;
+        l += __shfl_xor_sync(FULL, l, 1);
+        l += __shfl_xor_sync(FULL, l, 2);
+        const bool complete = began && (m.flags & F_UNIT_END);
+        const size_t unit = (size_t)m.s * Hkv + m.h;
+        uint16_t* out_row = a.out + ((size_t)m.s * Hq + (size_t)m.h * G + g_row) * D + 2 * c4;
+        if (complete) {
+            if (g_row < G) {
+                const float inv = 1.0f / l;
+#pragma unroll
+                for (int n = 0; n < D / 8; ++n)
+                    *reinterpret_cast<uint32_t*>(out_row + 8 * n) =
+                        pack_bf16x2(ws.o[n][0] * inv, ws.o[n][1] * inv);
+            }
+            return;
+        }
+        const long long nt = (m.len + TILE - 1) / TILE;
+        const long long au = m.f - m.t;                    // the unit's first flat tile
+        const long long bu = au + nt;
+        const int slot = (au < sc.begin(m.r)) ? 0 : 1;     // 0: the unit began in an earlier range
+        const size_t pbase = ((size_t)m.r * 2 + slot) * G;
+        if (g_row < G) {
+            float* po = a.part_o + (pbase + g_row) * D + 2 * c4;
+#pragma unroll
+            for (int n = 0; n < D / 8; ++n)
+                st_cg(reinterpret_cast<float2*>(po + 8 * n), make_float2(ws.o[n][0], ws.o[n][1]));
+            if (c4 == 0) st_cg(a.part_mz + pbase + g_row, make_float2(ws.m, l));
+        }
+        __threadfence();
+        __syncwarp();
+        const long long r_lo = sc.range_of(au);
+        const long long r_hi = sc.range_of(bu - 1);
+        unsigned prev = 0;
+        if (lane == 0) prev = atomicAdd(a.tickets + unit, 1u);
+        prev = __shfl_sync(FULL, prev, 0);
+        if (prev != (unsigned)(r_hi - r_lo)) return;      // not the last piece
+        __threadfence();
+        if (lane == 0) st_cg(reinterpret_cast<int*>(a.tickets) + unit, 0);   // ready for the next launch
+        // merge every piece of this unit (max-rescaled), in range order
+        float M[G], den[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) { M[g] = -INFINITY; den[g] = 0.f; }
+        for (long long j = r_lo; j <= r_hi; ++j) {
+            const int sl = (au < sc.begin(j)) ? 0 : 1;
+#pragma unroll
+            for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], ld_cg(a.part_mz + ((size_t)j * 2 + sl) * G + g).x);
+        }
+        constexpr int V4 = G * D / 4;                       // float4 per piece
+        constexpr int PER = (V4 + 31) / 32;
+        float4 acc4[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+        for (long long j = r_lo; j <= r_hi; ++j) {
+            const int sl = (au < sc.begin(j)) ? 0 : 1;
+            const size_t jb = ((size_t)j * 2 + sl) * G;
+            float cf[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float2 mz = ld_cg(a.part_mz + jb + g);
+                cf[g] = fast_exp2(mz.x - M[g]);
+                den[g] = fmaf(cf[g], mz.y, den[g]);
+            }
+            const float4* po = reinterpret_cast<const float4*>(a.part_o + jb * D);
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int e = lane + 32 * i;
+                if (e < V4) {
+                    const float4 v = ld_cg(po + e);
+                    const float cg = pick<G>(cf, (e * 4) / D);
+                    acc4[i].x = fmaf(cg, v.x, acc4[i].x);
+                    acc4[i].y = fmaf(cg, v.y, acc4[i].y);
+                    acc4[i].z = fmaf(cg, v.z, acc4[i].z);
+                    acc4[i].w = fmaf(cg, v.w, acc4[i].w);
+                }
+            }
+        }
+        uint16_t* o = a.out + ((size_t)m.s * Hq + (size_t)m.h * G) * D;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane + 32 * i;
+            if (e < V4) {
+                const float inv = 1.0f / pick<G>(den, (e * 4) / D);
+                uint2 pk;
+                pk.x = pack_bf16x2(acc4[i].x * inv, acc4[i].y * inv);
+                pk.y = pack_bf16x2(acc4[i].z * inv, acc4[i].w * inv);
+                *reinterpret_cast<uint2*>(o + (size_t)e * 4) = pk;
+            }
+        }
+    };
+
+    // ---- main loop ------------------------------------------------------------------
+    int issued = 0;
+    bool more = have_work;
+    while (issued < STAGES && more) {
+        more = issue(issued);
+        if (more) ++issued;
+    }
+    int failed_at = -1;
+    for (int i = 0; i < issued; ++i) {
+        const int st = i % STAGES;
+        const bool ok = mbar_wait_bounded(smem_addr(&bars[st]), (uint32_t)(i / STAGES) & 1u,
+                                          WAIT_LIMIT_NS);
+        if (__any_sync(FULL, !ok)) { failed_at = i; break; }
+        const StageMeta m = meta[st];
+        unsigned char* sKp = ring + (size_t)st * C::STAGE_BYTES;
+        const uint32_t sK = smem_addr(sKp);
+        const uint32_t sV = sK + C::KT_BYTES;
+        if (m.flags & F_FIRST) {
+            load_q_frags<D, G>(qa, reinterpret_cast<const uint16_t*>(qslots + (size_t)st * C::Q_BYTES),
+                               lane);
+            ws.reset();
+            began = (m.flags & F_UNIT_START) != 0;
+        }
+        const int nv = min(TILE, m.len - m.t * TILE);
+        if (nv < TILE) {
+            // zero the V rows past the sequence's end (0 * NaN would poison P V)
+            unsigned char* vbase = sKp + C::KT_BYTES;
+            for (int e = lane; e < (TILE - nv) * TS::HALVES * 8; e += 32) {
+                const int row = nv + e / (TS::HALVES * 8);
+                const int rest = e % (TS::HALVES * 8);
+                *reinterpret_cast<uint4*>(vbase + TS::row_offset(row, rest >> 3) + ((rest & 7) << 4)) =
+                    make_uint4(0, 0, 0, 0);
+            }
+            __syncwarp();
+            mma_tile<D, BS, true>(ws, qa, sK, sV, nv, a.qscale, lane);
+        } else {
+            mma_tile<D, BS, false>(ws, qa, sK, sV, nv, a.qscale, lane);
+        }
+        if (m.flags & F_LAST) finish_unit(m);
+        __syncwarp();
+        if (more) {
+            more = issue(st);
+            if (more) ++issued;
+        }
+    }
+    if (failed_at >= 0) {
+        if (lane == 0) raise_status(PKV_DEV_TIMEOUT);
+        for (int i = failed_at; i < issued; ++i)
+            mbar_wait_bounded(smem_addr(&bars[i % STAGES]), (uint32_t)(i / STAGES) & 1u,
+                              DRAIN_LIMIT_NS);
+    }
+}
+
+}  // namespace pkv

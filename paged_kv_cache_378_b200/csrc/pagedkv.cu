@@ -1,22 +1,34 @@
 // Host side of the C ABI declared in include/pagedkv.h: argument checks,
 // launch shapes and template dispatch.  Every entry point launches on the
 // caller's stream and never synchronises (except pkv_get_device_status).
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "pagedkv.h"
 #include "pkv_device.cuh"
 #include "kv_append.cuh"
 #include "block_copy.cuh"
-#include "paged_attention.cuh"
+#include "attn_paged.cuh"
 
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kAttnWarps = 4;
+// Attention CTA shape: warps per CTA and pipeline stages per warp (build-time
+// tunables; the stage count is per head_dim / block size, see attn_stages).
+#ifndef PKV_ATTN_WARPS
+#define PKV_ATTN_WARPS 4
+#endif
+#ifndef PKV_ATTN_STAGE_BUDGET
+#define PKV_ATTN_STAGE_BUDGET 8192    // bytes of K+V tiles per warp ring
+#endif
+constexpr int kAttnWarps = PKV_ATTN_WARPS;
+constexpr int kMaxCtasPerSm = 16;
 
 int device_sm_count() {
     static int cached[kMaxDevices] = {0};
@@ -34,7 +46,7 @@ int device_sm_count() {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool supported_head_dim(int d) { return d == 64 || d == 128; }
-bool supported_block_size(int b) { return b == 8 || b == 16 || b == 32; }
+bool supported_block_size(int b) { return b == 4 || b == 8 || b == 16 || b == 32; }
 
 int check_cache(const pkv_cache_t* c) {
     if (!c || !c->k_pool || !c->v_pool) return PKV_ERR_NULL;
@@ -56,94 +68,163 @@ int launch_status() {
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
-int tile_tokens(int block_size) { return block_size < 16 ? 16 : block_size; }
+// tokens per pipeline stage of the attention kernel (TileSmem::TILE)
+int tile_tokens(int head_dim, int block_size) {
+    return block_size >= 32 ? block_size : ((head_dim == 64 && block_size >= 8) ? 32 : 16);
+}
 
-// KV partition length.  Default: 256 tokens, grown while a launch would
-// still have more than 16 CTAs per SM at full length, so long sequences are
-// split across SMs while short-sequence batches keep few partitions.
-int resolve_partition(int num_seqs, int num_kv_heads, int max_blocks, int block_size,
-                      int requested) {
-    if (num_seqs < 0 || num_kv_heads <= 0 || max_blocks <= 0 || !supported_block_size(block_size))
-        return -1;
-    const int tile = tile_tokens(block_size);
-    long long pt;
-    if (requested > 0) {
-        pt = requested;
-    } else {
-        const long long max_len = (long long)max_blocks * block_size;
-        const long long units = (long long)num_seqs * num_kv_heads;
-        const long long sms = device_sm_count();
-        pt = 256;
-        while (pt < 4096 && units * ((max_len + pt - 1) / pt) > 16 * sms) pt *= 2;
-    }
-    pt = (pt + tile - 1) / tile * tile;
-    if (pt > (1LL << 30)) return -1;
-    return (int)pt;
+// Longest work range, in tokens, rounded up to the tile; 0 = no cap (ranges
+// are as long as an even split of the whole batch over the grid's warps).
+int resolve_partition(int head_dim, int block_size, int requested) {
+    if (!supported_block_size(block_size) || !supported_head_dim(head_dim) || requested < 0) return -1;
+    if (requested == 0) return 0;
+    const long long tile = tile_tokens(head_dim, block_size);
+    const long long pt = ((long long)requested + tile - 1) / tile * tile;
+    return pt > (1LL << 30) ? -1 : (int)pt;
+}
+
+template <int D, int BS>
+constexpr int attn_stages() {
+    return PKV_ATTN_STAGE_BUDGET / (2 * pkv::TileSmem<D, BS>::KT_BYTES) < 2
+               ? 2
+               : PKV_ATTN_STAGE_BUDGET / (2 * pkv::TileSmem<D, BS>::KT_BYTES);
 }
 
 struct WorkspaceLayout {
-    size_t o_off, mz_off, cnt_off, total;
-    int partitions;
+    size_t prefix_off, mz_off, o_off, tickets_off, total;
+    int R_max;
+    int cap_tiles;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// The tile prefix of large batches, two partials per range (one warp of the
+// largest grid this device can run is one range; a cap adds one range per
+// cap-length piece of the longest possible batch), one ticket per
+// (sequence, kv head).
 bool workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                       int max_blocks, int block_size, int partition_tokens, WorkspaceLayout* w) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
         !supported_head_dim(head_dim) || max_blocks <= 0 || !supported_block_size(block_size))
         return false;
-    const int pt = resolve_partition(num_seqs, num_kv_heads, max_blocks, block_size, partition_tokens);
-    if (pt <= 0) return false;
-    const long long max_len = (long long)max_blocks * block_size;
-    const int parts = (int)((max_len + pt - 1) / pt);
-    const size_t units = (size_t)num_seqs * num_kv_heads;
+    const int pt = resolve_partition(head_dim, block_size, partition_tokens);
+    if (pt < 0) return false;
+    const int tile = tile_tokens(head_dim, block_size);
+    const long long max_tiles = ((long long)max_blocks * block_size + tile - 1) / tile;
+    long long r_max = (long long)device_sm_count() * kMaxCtasPerSm * kAttnWarps;
+    const int cap_tiles = pt / tile;
+    if (cap_tiles > 0)
+        r_max += ((long long)num_seqs * num_kv_heads * max_tiles + cap_tiles - 1) / cap_tiles + 1;
+    if (r_max > (1LL << 30)) return false;
     const size_t G = (size_t)(num_q_heads / num_kv_heads);
-    w->partitions = parts;
-    w->o_off = 0;
-    w->mz_off = align_up(units * parts * G * head_dim * sizeof(float), 256);
-    w->cnt_off = w->mz_off + align_up(units * parts * G * sizeof(float2), 256);
-    w->total = w->cnt_off + align_up(units * sizeof(unsigned int), 256);
+    const size_t N = (size_t)num_seqs;
+    w->R_max = (int)r_max;
+    w->cap_tiles = cap_tiles;
+    w->prefix_off = 0;
+    w->mz_off = N > (size_t)pkv::PREFIX_SMEM ? align_up((N + 1) * sizeof(long long), 256) : 0;
+    w->o_off = w->mz_off + align_up((size_t)r_max * 2 * G * sizeof(float2), 256);
+    w->tickets_off = w->o_off + align_up((size_t)r_max * 2 * G * head_dim * sizeof(float), 256);
+    w->total = w->tickets_off + align_up(N * num_kv_heads * sizeof(unsigned int), 256);
     return true;
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (no link-time dependency on libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D view of a whole pool (all layers): rows of head_dim bf16, one TMA box =
+// one (block, kv head) tile's block_size rows x 64 dims, 128-byte swizzle.
+bool encode_pool_map(CUtensorMap* map, void* pool, const pkv_cache_t* c) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const unsigned long long rows =
+        (unsigned long long)c->num_layers * c->num_blocks * c->num_kv_heads * c->block_size;
+    if (rows > (1ull << 31)) return false;   // row coordinates are 32-bit signed
+    const cuuint64_t dims[2] = {(cuuint64_t)c->head_dim, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)c->head_dim * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)c->block_size};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pool, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// One template instance of the attention kernel: configuration, occupancy and launch.
 template <int D, int G, int BS>
-int launch_attention(const pkv::AttnArgs& args, int num_seqs, cudaStream_t s) {
-    using C = pkv::AttnCfg<D, G, BS, kAttnWarps>;
-    auto kern = pkv::paged_attention_kernel<D, G, BS, kAttnWarps>;
-    static bool configured[kMaxDevices] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-            cudaSuccess)
-            return PKV_ERR_CUDA;
-        configured[dev] = true;
+struct Attn {
+    static constexpr int STAGES = attn_stages<D, BS>();
+    using C = pkv::AttnCfg<D, G, BS, kAttnWarps, STAGES>;
+
+    static int ctas_per_sm() {
+        static int cached[kMaxDevices] = {0};
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+        if (cached[dev] == 0) {
+            auto kern = pkv::paged_attention_kernel<D, G, BS, kAttnWarps, STAGES>;
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+                cudaSuccess)
+                return -1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kAttnWarps * 32, C::SMEM_BYTES) !=
+                    cudaSuccess || n <= 0)
+                return -1;
+            cached[dev] = n < kMaxCtasPerSm ? n : kMaxCtasPerSm;
+        }
+        return cached[dev];
     }
-    const dim3 grid(args.num_partitions, args.num_kv_heads, num_seqs);
-    kern<<<grid, kAttnWarps * 32, C::SMEM_BYTES, s>>>(args);
-    return launch_status();
+
+    static int launch(const CUtensorMap& mk, const CUtensorMap& mv, const pkv::AttnArgs& a, int grid,
+                      cudaStream_t s) {
+        pkv::paged_attention_kernel<D, G, BS, kAttnWarps, STAGES>
+            <<<grid, kAttnWarps * 32, C::SMEM_BYTES, s>>>(mk, mv, a);
+        return launch_status();
+    }
+};
+
+// Dispatch on (head_dim, group, block size); op(Attn<...>{}) for the instance.
+template <typename Op>
+int with_instance(int D, int G, int BS, Op&& op) {
+#define PKV_BS(DD, GG)                                             \
+    switch (BS) {                                                  \
+        case 4: return op(Attn<DD, GG, 4>{});                      \
+        case 8: return op(Attn<DD, GG, 8>{});                      \
+        case 16: return op(Attn<DD, GG, 16>{});                    \
+        case 32: return op(Attn<DD, GG, 32>{});                    \
+    }                                                              \
+    return PKV_ERR_UNSUPPORTED;
+#define PKV_G(DD)                                                  \
+    switch (G) {                                                   \
+        case 1: { PKV_BS(DD, 1) }                                  \
+        case 2: { PKV_BS(DD, 2) }                                  \
+        case 4: { PKV_BS(DD, 4) }                                  \
+        case 8: { PKV_BS(DD, 8) }                                  \
+    }                                                              \
+    return PKV_ERR_UNSUPPORTED;
+    if (D == 64) { PKV_G(64) }
+    if (D == 128) { PKV_G(128) }
+    return PKV_ERR_UNSUPPORTED;
+#undef PKV_G
+#undef PKV_BS
 }
 
-template <int D, int G>
-int dispatch_block(int bs, const pkv::AttnArgs& a, int n, cudaStream_t s) {
-    switch (bs) {
-        case 8: return launch_attention<D, G, 8>(a, n, s);
-        case 16: return launch_attention<D, G, 16>(a, n, s);
-        case 32: return launch_attention<D, G, 32>(a, n, s);
-    }
-    return PKV_ERR_UNSUPPORTED;
-}
-
-template <int D>
-int dispatch_group(int g, int bs, const pkv::AttnArgs& a, int n, cudaStream_t s) {
-    switch (g) {
-        case 1: return dispatch_block<D, 1>(bs, a, n, s);
-        case 2: return dispatch_block<D, 2>(bs, a, n, s);
-        case 4: return dispatch_block<D, 4>(bs, a, n, s);
-        case 8: return dispatch_block<D, 8>(bs, a, n, s);
-    }
-    return PKV_ERR_UNSUPPORTED;
+// Warps of the attention grid for this instance on the current device.
+int grid_warps_for(int D, int G, int BS) {
+    const int n = with_instance(D, G, BS, [](auto inst) { return decltype(inst)::ctas_per_sm(); });
+    const int per_sm = n > 0 ? n : kMaxCtasPerSm;
+    return device_sm_count() * per_sm * kAttnWarps;
 }
 
 }  // namespace
@@ -208,13 +289,14 @@ int pkv_block_copy(const pkv_cache_t* cache, const int32_t* src_dst_pairs, int n
 
 int pkv_partition_tokens(int num_seqs, int num_kv_heads, int head_dim, int max_blocks_per_seq,
                          int block_size, int requested) {
-    if (!supported_head_dim(head_dim) || requested < 0) return -1;
-    return resolve_partition(num_seqs, num_kv_heads, max_blocks_per_seq, block_size, requested);
+    if (!supported_head_dim(head_dim) || num_seqs < 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0)
+        return -1;
+    return resolve_partition(head_dim, block_size, requested);
 }
 
 size_t pkv_attention_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                      int max_blocks_per_seq, int block_size, int partition_tokens) {
-    if (partition_tokens < 0) return 0;
+    if (num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads) return 0;
     WorkspaceLayout w;
     if (!workspace_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                           block_size, partition_tokens, &w))
@@ -244,39 +326,44 @@ int pkv_paged_decode_attention(const pkv_cache_t* cache, int layer, const void* 
     const int G = num_q_heads / cache->num_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return PKV_ERR_UNSUPPORTED;
     if (num_seqs == 0) return PKV_OK;
-    if (num_seqs > 65535 || cache->num_kv_heads > 65535) return PKV_ERR_SHAPE;
+    if ((long long)max_blocks_per_seq * cache->block_size > (1LL << 30)) return PKV_ERR_SHAPE;
     if (!q || !block_tables || !seq_lens || !out) return PKV_ERR_NULL;
     if (!aligned16(q) || !aligned16(out)) return PKV_ERR_ALIGN;
+    const int D = cache->head_dim, BS = cache->block_size;
+    const int grid_warps = grid_warps_for(D, G, BS);
     WorkspaceLayout w;
-    if (!workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, cache->head_dim,
-                          max_blocks_per_seq, cache->block_size, partition_tokens, &w))
+    if (!workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, D, max_blocks_per_seq, BS,
+                          partition_tokens, &w))
         return PKV_ERR_SHAPE;
-    if (w.partitions > 1) {
-        if (!workspace) return PKV_ERR_WORKSPACE;
-        if (workspace_bytes < w.total || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
-    }
+    if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
+    if (grid_warps > w.R_max) return PKV_ERR_WORKSPACE;
+
+    CUtensorMap mk, mv;
+    if (!encode_pool_map(&mk, cache->k_pool, cache) || !encode_pool_map(&mv, cache->v_pool, cache))
+        return PKV_ERR_CUDA;
     pkv::AttnArgs a;
-    const size_t base = (size_t)layer * layer_elems(cache);
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
     a.q = static_cast<const uint16_t*>(q);
-    a.k_pool = static_cast<const uint16_t*>(cache->k_pool) + base;
-    a.v_pool = static_cast<const uint16_t*>(cache->v_pool) + base;
     a.out = static_cast<uint16_t*>(out);
     a.block_tables = block_tables;
     a.seq_lens = seq_lens;
-    unsigned char* ws = static_cast<unsigned char*>(workspace);
-    a.part_o = ws ? reinterpret_cast<float*>(ws + w.o_off) : nullptr;
-    a.part_mz = ws ? reinterpret_cast<float2*>(ws + w.mz_off) : nullptr;
-    a.counters = ws ? reinterpret_cast<unsigned int*>(ws + w.cnt_off) : nullptr;
+    a.num_seqs = num_seqs;
     a.num_kv_heads = cache->num_kv_heads;
     a.num_blocks = cache->num_blocks;
     a.max_blocks = max_blocks_per_seq;
-    a.partition_tokens = resolve_partition(num_seqs, cache->num_kv_heads, max_blocks_per_seq,
-                                           cache->block_size, partition_tokens);
-    a.num_partitions = w.partitions;
     a.qscale = (float)((double)scale * 1.4426950408889634074);   // scale * log2(e)
+    a.row_base = (long long)layer * cache->num_blocks * cache->num_kv_heads * cache->block_size;
+    a.part_mz = reinterpret_cast<float2*>(ws + w.mz_off);
+    a.part_o = reinterpret_cast<float*>(ws + w.o_off);
+    a.tickets = reinterpret_cast<unsigned int*>(ws + w.tickets_off);
+    a.prefix_g = reinterpret_cast<long long*>(ws + w.prefix_off);
+    a.R_max = w.R_max;
+    a.cap_tiles = w.cap_tiles;
+    a.K = grid_warps;
     cudaStream_t s = (cudaStream_t)stream;
-    if (cache->head_dim == 64) return dispatch_group<64>(G, cache->block_size, a, num_seqs, s);
-    return dispatch_group<128>(G, cache->block_size, a, num_seqs, s);
+    return with_instance(D, G, BS, [&](auto inst) {
+        return decltype(inst)::launch(mk, mv, a, grid_warps / kAttnWarps, s);
+    });
 }
 
 int pkv_get_device_status(unsigned int* status_out, int reset) {

@@ -60,7 +60,7 @@ def test_host_argument_checks_before_launch():
     assert lib.pkv_block_copy(P(_cache(k_pool=0)), 16, 1, None) == -1
     # unsupported shapes
     assert lib.pkv_kv_append(P(_cache(head_dim=96)), 0, 16, 16, 16, 1, None) == -5
-    assert lib.pkv_kv_append(P(_cache(block_size=4)), 0, 16, 16, 16, 1, None) == -5
+    assert lib.pkv_kv_append(P(_cache(block_size=12)), 0, 16, 16, 16, 1, None) == -5
     assert lib.pkv_kv_append(P(_cache(num_blocks=0)), 0, 16, 16, 16, 1, None) == -2
     # misaligned pool / inputs
     assert lib.pkv_kv_append(P(_cache(k_pool=18)), 0, 16, 16, 16, 1, None) == -3
@@ -80,7 +80,7 @@ def test_host_argument_checks_before_launch():
     assert att(P(c), 0, 16, 0, 8, 16, 4, 16, 0.125, 16, None, 0, 0, None) == 0
     assert att(P(c), 0, None, 2, 8, 16, 4, 16, 0.125, 16, None, 0, 0, None) == -1
     assert att(P(c), 0, 16, 2, 8, 16, 4, 16, 0.125, 40, None, 0, 0, None) == -3
-    # a table that spans several partitions needs a workspace of the right size
+    # the workspace is required and must be large enough
     assert att(P(c), 0, 16, 2, 8, 16, 4096, 16, 0.125, 16, None, 0, 512, None) == -4
     need = lib.pkv_attention_workspace_bytes(2, 8, 2, 64, 4096, 16, 512)
     assert need > 0
@@ -89,17 +89,27 @@ def test_host_argument_checks_before_launch():
 
 def test_workspace_and_partition_sizes():
     lib = pkv.library()
-    # partition rounds up to the tile (16 tokens, or the block when larger)
+    # a requested partition rounds up to the tile: 32 tokens at head_dim 64 (16 with
+    # 4-token blocks), 16 at head_dim 128, never less than one block
     assert lib.pkv_partition_tokens(8, 8, 128, 2048, 16, 500) == 512
     assert lib.pkv_partition_tokens(8, 8, 128, 2048, 32, 40) == 64
-    assert lib.pkv_partition_tokens(8, 8, 64, 2048, 8, 1) == 16
+    assert lib.pkv_partition_tokens(8, 8, 64, 2048, 8, 1) == 32
+    assert lib.pkv_partition_tokens(8, 8, 64, 2048, 16, 33) == 64
+    assert lib.pkv_partition_tokens(8, 8, 64, 2048, 4, 20) == 32
     assert lib.pkv_partition_tokens(8, 8, 96, 2048, 8, 1) == -1
-    d = lib.pkv_partition_tokens(64, 8, 64, 128, 16, 0)
-    assert d >= 256 and d % 16 == 0
-    # bytes grow with the number of partitions: (G*d + G*2) floats per partition + counters
+    assert lib.pkv_partition_tokens(64, 8, 64, 128, 16, 0) == 0      # no cap: even split
+    # the workspace holds two partials per range (one range per warp of the grid,
+    # more under a cap): (m, Z) + d floats for each of G heads, and a ticket per
+    # (sequence, kv head); a cap of C tokens adds ceil(N*Hkv*max_tiles / C) ranges
+    n0 = lib.pkv_attention_workspace_bytes(8, 32, 8, 128, 2048, 16, 0)
     n1 = lib.pkv_attention_workspace_bytes(8, 32, 8, 128, 2048, 16, 512)
-    parts = 32768 // 512
     units = 8 * 8
-    assert n1 >= units * parts * 4 * (128 + 2) * 4 + units * 4
+    per_range = 2 * 4 * (2 + 128) * 4
+    assert n0 >= 148 * 4 * per_range + units * 4
+    assert n1 - n0 >= (units * 2048 // 32) * per_range
+    # more than 1024 sequences: the tile prefix lives in the workspace too
+    big = lib.pkv_attention_workspace_bytes(2048, 32, 8, 64, 16, 16, 0)
+    small = lib.pkv_attention_workspace_bytes(1024, 32, 8, 64, 16, 16, 0)
+    assert big - small >= 2049 * 8
     assert lib.pkv_attention_workspace_bytes(8, 30, 8, 128, 2048, 16, 512) == 0
     assert lib.pkv_attention_workspace_bytes(8, 32, 8, 128, 2048, 12, 512) == 0

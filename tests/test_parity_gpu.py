@@ -156,7 +156,7 @@ def _custom(D, G, B, N=6, lens="uniform:1,300", seed=0):
 
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
-@pytest.mark.parametrize("B", [8, 16, 32])
+@pytest.mark.parametrize("B", [4, 8, 16, 32])
 def test_shape_sweep_with_split_partitions(D, G, B):
     spec = _custom(D, G, B, seed=100 + D + 10 * G + B)
     w = make_workload(spec)
@@ -167,7 +167,10 @@ def test_shape_sweep_with_split_partitions(D, G, B):
         assert_close(f64(outs[0]), ref, f"D={D} G={G} B={B} part={part}")
 
 
-def test_physical_permutation_gives_identical_bits():
+def test_physical_permutation_invariance():
+    """Relabelling physical blocks changes nothing: both runs match the oracle
+    and are bit-identical (the work split depends only on the lengths, and
+    split pieces are merged in a fixed order)."""
     w = make_workload("continuous_batch")
     out1 = gpu_step(pkv, w, device_inputs(w))[0]
     perm = np.random.default_rng(3).permutation(w.num_blocks)
@@ -185,6 +188,9 @@ def test_physical_permutation_gives_identical_bits():
     blk, off = np.divmod(w.slot_mapping, w.block_size)
     w2.slot_mapping = perm[blk] * w.block_size + off
     out2 = gpu_step(pkv, w2, device_inputs(w2))[0]
+    ref = _oracle_attention(w, 0)
+    assert_close(f64(out1), ref, "original ids")
+    assert_close(f64(out2), ref, "permuted ids")
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
 
 
@@ -195,12 +201,14 @@ def test_workspace_reuse_is_stable():
     ws = pkv.make_workspace(w.num_seqs, spec.num_q_heads, spec.num_kv_heads, spec.head_dim,
                             w.max_blocks, w.block_size, 512)
     a = gpu_step(pkv, w, dev, workspace=ws)[0].clone()
+    ref = _oracle_attention(w, 0)
+    assert_close(f64(a), ref, "first call")
     for _ in range(3):
         b = gpu_step(pkv, w, dev, workspace=ws)[0]
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     # every split-K counter is back at zero
-    # every split-K counter (the workspace's last 256 bytes here: 64 counters) is back at zero
-    assert w.num_seqs * spec.num_kv_heads * 4 <= 256
+    # every ticket (the workspace's last 256 bytes here: 64 of them) is back at zero
+    assert w.num_seqs * spec.num_kv_heads * 4 == 256
     assert int(ws[-256:].view(torch.int32).abs().sum()) == 0
     _assert_no_device_error()
 
