@@ -43,7 +43,7 @@ UNIT = "GB/s"
 DEFAULT_WORKLOAD = "continuous_batch"
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "attention_traffic.json")
-KERNEL_SOURCES = ["pkv_device.cuh", "paged_attention.cuh", "pagedkv.cu"]
+KERNEL_SOURCES = ["pkv_device.cuh", "attn_common.cuh", "attn_paged.cuh", "pagedkv.cu"]
 
 
 # ---------------------------------------------------------------------------
