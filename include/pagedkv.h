@@ -63,6 +63,10 @@ extern "C" {
 #define PKV_ERR_UNSUPPORTED  -5  /* head_dim / block_size / group size not built */
 #define PKV_ERR_CUDA         -6  /* a CUDA runtime call or launch failed */
 #define PKV_ERR_LAYER        -7  /* layer index outside [0, num_layers) */
+#define PKV_ERR_SCRATCH      -8  /* request too large for the no-allocation scratch */
+
+/* size of the device buffer behind pkv_paged_decode_attention_noalloc */
+#define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
 
 /* device-side status bits (pkv_get_device_status) */
 #define PKV_DEV_RANGE    0x1u  /* block id or slot outside the pool: access skipped */
@@ -191,6 +195,43 @@ int pkv_paged_decode_attention(const pkv_cache_t* cache, int layer,
                                const int32_t* seq_lens, float scale, void* out,
                                void* workspace, size_t workspace_bytes,
                                int partition_tokens, void* stream);
+
+/*
+ * pkv_paged_decode_attention_noalloc -- pkv_paged_decode_attention for callers
+ * that cannot allocate device memory.  The pages describe no such call.  It is
+ * for code that has no way to get a workspace: a plugin inside a host
+ * framework that owns all device memory and hands the plugin only its input
+ * and output buffers, or a real-time serving loop that must never call the
+ * allocator (an allocation can fail, or synchronise the device, at the worst
+ * moment).
+ *
+ * Same arguments and result as pkv_paged_decode_attention, without a
+ * workspace: the scratch (partial results of split sequences, one ticket per
+ * (sequence, kv head), the tile prefix of batches over 1024 sequences) lives
+ * in one fixed device array of PKV_NOALLOC_SCRATCH_BYTES (16 MiB) inside this
+ * library.  Every GPU that loads the library holds that array until the
+ * process exits.  The call itself allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ *
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and keeps it; make that
+ *     first call before any stream capture.
+ *   - Each call zeroes the tickets it uses (an asynchronous memset on
+ *     `stream`), then launches the attention kernel on `stream`.
+ *   - All calls share the one array and it keeps the last call's contents:
+ *     calls whose GPU work can overlap (different streams without ordering
+ *     between them, or concurrent host threads on different streams) race
+ *     and give wrong results.  Order them on one stream.
+ *   - A request whose scratch would exceed PKV_NOALLOC_SCRATCH_BYTES returns
+ *     PKV_ERR_SCRATCH before launching anything (the size grows with the
+ *     number of warps the device runs, the group size G, head_dim, and with
+ *     a partition cap, the batch's total length).
+ */
+int pkv_paged_decode_attention_noalloc(const pkv_cache_t* cache, int layer,
+                                       const void* q, int num_seqs, int num_q_heads,
+                                       const int32_t* block_tables, int max_blocks_per_seq,
+                                       const int32_t* seq_lens, float scale, void* out,
+                                       int partition_tokens, void* stream);
 
 /*
  * pkv_get_device_status -- read (and with reset != 0, clear) the device status

@@ -227,6 +227,58 @@ int grid_warps_for(int D, int G, int BS) {
     return device_sm_count() * per_sm * kAttnWarps;
 }
 
+// ---- attention without allocation ------------------------------------------
+//
+// Scratch for pkv_paged_decode_attention_noalloc: one fixed array per device
+// that loads this library, kept for the life of the process.  Host code must
+// not pass the array's name to a kernel (on the host it is only a stand-in
+// symbol); the device address comes from cudaGetSymbolAddress, taken once per
+// device on that device's first call.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PKV_NOALLOC_SCRATCH_BYTES];
+
+// Layout of the scratch for one call: the same regions as a caller-provided
+// workspace, sized for the grid this call launches rather than the largest
+// grid the device could run.
+bool noalloc_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_blocks,
+                    int block_size, int partition_tokens, int grid_warps, WorkspaceLayout* w) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
+        !supported_head_dim(head_dim) || max_blocks <= 0 || !supported_block_size(block_size) ||
+        grid_warps <= 0)
+        return false;
+    const int pt = resolve_partition(head_dim, block_size, partition_tokens);
+    if (pt < 0) return false;
+    const int tile = tile_tokens(head_dim, block_size);
+    const long long max_tiles = ((long long)max_blocks * block_size + tile - 1) / tile;
+    long long r_max = grid_warps;
+    const int cap_tiles = pt / tile;
+    if (cap_tiles > 0)
+        r_max += ((long long)num_seqs * num_kv_heads * max_tiles + cap_tiles - 1) / cap_tiles + 1;
+    if (r_max > (1LL << 30)) return false;
+    const size_t G = (size_t)(num_q_heads / num_kv_heads);
+    const size_t N = (size_t)num_seqs;
+    w->R_max = (int)r_max;
+    w->cap_tiles = cap_tiles;
+    w->prefix_off = 0;
+    w->mz_off = N > (size_t)pkv::PREFIX_SMEM ? align_up((N + 1) * sizeof(long long), 256) : 0;
+    w->o_off = w->mz_off + align_up((size_t)r_max * 2 * G * sizeof(float2), 256);
+    w->tickets_off = w->o_off + align_up((size_t)r_max * 2 * G * head_dim * sizeof(float), 256);
+    w->total = w->tickets_off + align_up(N * num_kv_heads * sizeof(unsigned int), 256);
+    return true;
+}
+
+// Device address of the scratch on the current device (set up on first use).
+unsigned char* noalloc_scratch_ptr() {
+    static unsigned char* ptrs[kMaxDevices] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+        ptrs[dev] = static_cast<unsigned char*>(p);
+    }
+    return ptrs[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -243,6 +295,9 @@ const char* pkv_strerror(int code) {
         case PKV_ERR_UNSUPPORTED: return "head_dim / block_size / group size not supported";
         case PKV_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
         case PKV_ERR_LAYER: return "layer index outside the cache";
+        case PKV_ERR_SCRATCH:
+            return "request needs more scratch than the no-allocation buffer holds "
+                   "(PKV_NOALLOC_SCRATCH_BYTES); use pkv_paged_decode_attention with a workspace";
     }
     return "unknown pagedkv status";
 }
@@ -361,6 +416,63 @@ int pkv_paged_decode_attention(const pkv_cache_t* cache, int layer, const void* 
     a.cap_tiles = w.cap_tiles;
     a.K = grid_warps;
     cudaStream_t s = (cudaStream_t)stream;
+    return with_instance(D, G, BS, [&](auto inst) {
+        return decltype(inst)::launch(mk, mv, a, grid_warps / kAttnWarps, s);
+    });
+}
+
+int pkv_paged_decode_attention_noalloc(const pkv_cache_t* cache, int layer, const void* q,
+                                       int num_seqs, int num_q_heads, const int32_t* block_tables,
+                                       int max_blocks_per_seq, const int32_t* seq_lens, float scale,
+                                       void* out, int partition_tokens, void* stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (layer < 0 || layer >= cache->num_layers) return PKV_ERR_LAYER;
+    if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || partition_tokens < 0)
+        return PKV_ERR_SHAPE;
+    if (num_q_heads % cache->num_kv_heads) return PKV_ERR_SHAPE;
+    if (!std::isfinite(scale)) return PKV_ERR_SHAPE;
+    const int G = num_q_heads / cache->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PKV_OK;
+    if ((long long)max_blocks_per_seq * cache->block_size > (1LL << 30)) return PKV_ERR_SHAPE;
+    if (!q || !block_tables || !seq_lens || !out) return PKV_ERR_NULL;
+    if (!aligned16(q) || !aligned16(out)) return PKV_ERR_ALIGN;
+    const int D = cache->head_dim, BS = cache->block_size;
+    const int grid_warps = grid_warps_for(D, G, BS);
+    WorkspaceLayout w;
+    if (!noalloc_layout(num_seqs, num_q_heads, cache->num_kv_heads, D, max_blocks_per_seq, BS,
+                        partition_tokens, grid_warps, &w))
+        return PKV_ERR_SHAPE;
+    if (w.total > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_ERR_SCRATCH;
+    unsigned char* ws = noalloc_scratch_ptr();
+    if (!ws) return PKV_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    // the tickets must start at zero; the scratch keeps whatever the last call left
+    const size_t ticket_bytes = (size_t)num_seqs * cache->num_kv_heads * sizeof(unsigned int);
+    if (cudaMemsetAsync(ws + w.tickets_off, 0, ticket_bytes, s) != cudaSuccess) return PKV_ERR_CUDA;
+
+    CUtensorMap mk, mv;
+    if (!encode_pool_map(&mk, cache->k_pool, cache) || !encode_pool_map(&mv, cache->v_pool, cache))
+        return PKV_ERR_CUDA;
+    pkv::AttnArgs a;
+    a.q = static_cast<const uint16_t*>(q);
+    a.out = static_cast<uint16_t*>(out);
+    a.block_tables = block_tables;
+    a.seq_lens = seq_lens;
+    a.num_seqs = num_seqs;
+    a.num_kv_heads = cache->num_kv_heads;
+    a.num_blocks = cache->num_blocks;
+    a.max_blocks = max_blocks_per_seq;
+    a.qscale = (float)((double)scale * 1.4426950408889634074);   // scale * log2(e)
+    a.row_base = (long long)layer * cache->num_blocks * cache->num_kv_heads * cache->block_size;
+    a.part_mz = reinterpret_cast<float2*>(ws + w.mz_off);
+    a.part_o = reinterpret_cast<float*>(ws + w.o_off);
+    a.tickets = reinterpret_cast<unsigned int*>(ws + w.tickets_off);
+    a.prefix_g = reinterpret_cast<long long*>(ws + w.prefix_off);
+    a.R_max = w.R_max;
+    a.cap_tiles = w.cap_tiles;
+    a.K = grid_warps;
     return with_instance(D, G, BS, [&](auto inst) {
         return decltype(inst)::launch(mk, mv, a, grid_warps / kAttnWarps, s);
     });
