@@ -191,6 +191,7 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int st = 0; st < STAGES; ++st) mbar_init(smem_addr(&bars[st]), 1);
         fence_mbar_init();
     }
+    pdl_wait();                                           // earlier kernels' writes are visible
 
     const int N = a.num_seqs;
     const int Hkv = a.num_kv_heads;
@@ -529,6 +530,10 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (more) ++issued;
         }
     }
+    // Let the next kernel on the stream start launching only now: its CTAs
+    // would otherwise sit resident (waiting) beside this kernel's warps for
+    // the whole launch.
+    pdl_launch_dependents();
     if (failed_at >= 0) {
         if (lane == 0) raise_status(PKV_DEV_TIMEOUT);
         for (int i = failed_at; i < issued; ++i)

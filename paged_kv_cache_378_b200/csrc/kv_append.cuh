@@ -16,6 +16,8 @@ kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_ne
                  uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,  // layer base
                  const int64_t* __restrict__ slot_mapping, int num_tokens,
                  int num_kv_heads, int block_size, int head_dim, int num_blocks) {
+    pdl_launch_dependents();
+    pdl_wait();                                          // earlier writes to the pool land first
     const int chunks_per_row = head_dim / 8;            // uint4 per head row
     const int chunks_per_tok = num_kv_heads * chunks_per_row;
     const long long total = (long long)num_tokens * chunks_per_tok * 2;

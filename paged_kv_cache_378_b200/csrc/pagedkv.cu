@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <utility>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -63,14 +64,32 @@ size_t layer_elems(const pkv_cache_t* c) {
     return (size_t)c->num_blocks * c->num_kv_heads * c->block_size * c->head_dim;
 }
 
-int launch_status() {
-    const cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
-}
-
 // tokens per pipeline stage of the attention kernel (TileSmem::TILE)
 int tile_tokens(int head_dim, int block_size) {
     return block_size >= 32 ? block_size : ((head_dim == 64 && block_size >= 8) ? 32 : 16);
+}
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on the stream finishes; every kernel here waits
+// (griddepcontrol.wait) before it reads or writes data.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+               Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
+        cudaGetLastError();
+        return PKV_ERR_CUDA;
+    }
+    return PKV_OK;
 }
 
 // Longest work range, in tokens, rounded up to the tile; 0 = no cap (ranges
@@ -188,9 +207,8 @@ struct Attn {
 
     static int launch(const CUtensorMap& mk, const CUtensorMap& mv, const pkv::AttnArgs& a, int grid,
                       cudaStream_t s) {
-        pkv::paged_attention_kernel<D, G, BS, kAttnWarps, STAGES>
-            <<<grid, kAttnWarps * 32, C::SMEM_BYTES, s>>>(mk, mv, a);
-        return launch_status();
+        return launch_pdl(pkv::paged_attention_kernel<D, G, BS, kAttnWarps, STAGES>, dim3(grid),
+                          dim3(kAttnWarps * 32), C::SMEM_BYTES, s, mk, mv, a);
     }
 };
 
@@ -317,12 +335,13 @@ int pkv_kv_append(const pkv_cache_t* cache, int layer, const void* k_new, const 
     long long blocks = (total + threads - 1) / threads;
     const long long cap = (long long)device_sm_count() * 16;
     if (blocks > cap) blocks = cap;
-    pkv::kv_append_kernel<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(
-        reinterpret_cast<const uint4*>(k_new), reinterpret_cast<const uint4*>(v_new),
-        reinterpret_cast<uint4*>(static_cast<uint16_t*>(cache->k_pool) + base),
-        reinterpret_cast<uint4*>(static_cast<uint16_t*>(cache->v_pool) + base), slot_mapping,
-        num_tokens, cache->num_kv_heads, cache->block_size, cache->head_dim, cache->num_blocks);
-    return launch_status();
+    return launch_pdl(pkv::kv_append_kernel, dim3((unsigned)blocks), dim3(threads), 0,
+                      (cudaStream_t)stream, reinterpret_cast<const uint4*>(k_new),
+                      reinterpret_cast<const uint4*>(v_new),
+                      reinterpret_cast<uint4*>(static_cast<uint16_t*>(cache->k_pool) + base),
+                      reinterpret_cast<uint4*>(static_cast<uint16_t*>(cache->v_pool) + base),
+                      slot_mapping, num_tokens, cache->num_kv_heads, cache->block_size,
+                      cache->head_dim, cache->num_blocks);
 }
 
 int pkv_block_copy(const pkv_cache_t* cache, const int32_t* src_dst_pairs, int num_pairs,
@@ -333,13 +352,13 @@ int pkv_block_copy(const pkv_cache_t* cache, const int32_t* src_dst_pairs, int n
     if (num_pairs == 0) return PKV_OK;
     if (!src_dst_pairs) return PKV_ERR_NULL;
     const long long chunks = (long long)cache->num_kv_heads * cache->block_size * cache->head_dim / 8;
-    long long units = (long long)num_pairs * cache->num_layers * 2;
+    const long long total = (long long)num_pairs * cache->num_layers * 2 * chunks;
+    const long long want = (total + 256 * 4 - 1) / (256 * 4);   // four chunks per thread
     const long long cap = (long long)device_sm_count() * 8;
-    const unsigned grid = (unsigned)(units < cap ? units : cap);
-    pkv::block_copy_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
-        reinterpret_cast<uint4*>(cache->k_pool), reinterpret_cast<uint4*>(cache->v_pool),
-        src_dst_pairs, num_pairs, cache->num_layers, cache->num_blocks, chunks);
-    return launch_status();
+    const unsigned grid = (unsigned)(want < cap ? want : cap);
+    return launch_pdl(pkv::block_copy_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream,
+                      reinterpret_cast<uint4*>(cache->k_pool), reinterpret_cast<uint4*>(cache->v_pool),
+                      src_dst_pairs, num_pairs, cache->num_layers, cache->num_blocks, chunks);
 }
 
 int pkv_partition_tokens(int num_seqs, int num_kv_heads, int head_dim, int max_blocks_per_seq,

@@ -25,6 +25,18 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// ---- programmatic dependent launch -------------------------------------------
+// pdl_wait: block until the kernels this grid depends on have completed and
+// their writes are visible (returns at once when launched without the
+// programmatic-serialization attribute).  pdl_launch_dependents: let the next
+// kernel on the stream start launching its CTAs; it still waits in pdl_wait
+// for this grid to finish before touching data.
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- mbarrier -------------------------------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
