@@ -212,6 +212,8 @@ class GpuStep:
         self.pairs = torch.from_numpy(w.copy_pairs).to(device)
         self.npairs = int(w.copy_pairs.shape[0])
         self.out = torch.empty_like(w.q)
+        self.resident = dict(q=self.q, k_new=self.k_new, v_new=self.v_new, tables=self.tables,
+                             lens=self.lens, slots=self.slots, pairs=self.pairs, out=self.out)
         self.partition = int(partition)
         self.ws = pkv.make_workspace(self.N, self.Hq, H, D, w.max_blocks, B, self.partition,
                                      device=device)
@@ -219,22 +221,25 @@ class GpuStep:
         self.maxb = w.max_blocks
         self.launches_per_step = (1 if self.npairs else 0) + 2 * self.L
 
-    def run(self, step_index, evl=None):
-        """Launch one step; ``evl`` = per-layer (start, end) events around attention."""
+    def run(self, step_index, evl=None, bufs=None):
+        """Launch one step; ``evl`` = per-layer (start, end) events around
+        attention; ``bufs`` = the step's input/output tensors (default: the
+        resident ones)."""
         lib = self.lib
+        b = bufs if bufs is not None else self.resident
         _, cref = self.caches[step_index % len(self.caches)]
         rc = 0
         if self.npairs:
-            rc |= lib.pkv_block_copy(cref, self.pairs.data_ptr(), self.npairs, self.sp)
+            rc |= lib.pkv_block_copy(cref, b["pairs"].data_ptr(), self.npairs, self.sp)
         for layer in range(self.L):
-            rc |= lib.pkv_kv_append(cref, layer, self.k_new[layer].data_ptr(),
-                                    self.v_new[layer].data_ptr(), self.slots.data_ptr(), self.N,
+            rc |= lib.pkv_kv_append(cref, layer, b["k_new"][layer].data_ptr(),
+                                    b["v_new"][layer].data_ptr(), b["slots"].data_ptr(), self.N,
                                     self.sp)
             if evl is not None:
                 evl[layer][0].record(self.stream)
             rc |= lib.pkv_paged_decode_attention(
-                cref, layer, self.q[layer].data_ptr(), self.N, self.Hq, self.tables.data_ptr(),
-                self.maxb, self.lens.data_ptr(), self.scale, self.out[layer].data_ptr(),
+                cref, layer, b["q"][layer].data_ptr(), self.N, self.Hq, b["tables"].data_ptr(),
+                self.maxb, b["lens"].data_ptr(), self.scale, b["out"][layer].data_ptr(),
                 self.ws.data_ptr(), self.ws.numel(), self.partition, self.sp)
             if evl is not None:
                 evl[layer][1].record(self.stream)
@@ -242,38 +247,79 @@ class GpuStep:
             raise RuntimeError(f"pagedkv call failed (status {rc})")
 
 
+def packed_buffers(like, device, pin):
+    """One contiguous byte buffer holding a tensor per entry of ``like`` (256-byte
+    aligned views), so a step's inputs move in a single copy."""
+    offs, total = {}, 0
+    for k, t in like.items():
+        offs[k] = total
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    raw = torch.empty(total, dtype=torch.uint8, device=device, pin_memory=pin)
+    views = {k: raw[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+             for (k, t), o in zip(like.items(), offs.values())}
+    return raw, views
+
+
 def e2e_run(pkv, w, gs, steps, device):
-    """Same step through the C ABI with host buffers: per step, H2D of the
-    step's inputs from pinned memory and D2H of the attention output."""
-    host = dict(q=w.q.cpu().pin_memory(), k_new=w.k_new.cpu().pin_memory(),
-                v_new=w.v_new.cpu().pin_memory(),
-                tables=torch.from_numpy(w.block_tables).pin_memory(),
-                lens=torch.from_numpy(w.seq_lens).pin_memory(),
-                slots=torch.from_numpy(w.slot_mapping).pin_memory(),
-                pairs=torch.from_numpy(w.copy_pairs).pin_memory())
-    out_host = torch.empty(gs.out.shape, dtype=gs.out.dtype).pin_memory()
-    dev_bufs = dict(q=gs.q, k_new=gs.k_new, v_new=gs.v_new, tables=gs.tables, lens=gs.lens,
-                    slots=gs.slots, pairs=gs.pairs)
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_host.numel() * out_host.element_size()
-    s = gs.stream
+    """The same step through the C ABI from host buffers.  Every step uploads
+    its inputs (q, k_new, v_new, block tables, lengths, slot mapping, copy
+    pairs: one packed pinned buffer, one copy) and reads its attention output
+    back to pinned host memory.  Two buffer sets alternate, so step i+1's
+    upload and step i-1's download run on copy streams while step i computes."""
+    host_src = dict(q=w.q.cpu(), k_new=w.k_new.cpu(), v_new=w.v_new.cpu(),
+                    tables=torch.from_numpy(w.block_tables), lens=torch.from_numpy(w.seq_lens),
+                    slots=torch.from_numpy(w.slot_mapping), pairs=torch.from_numpy(w.copy_pairs))
+    h_raw, h_views = packed_buffers(host_src, "cpu", True)
+    for k, t in host_src.items():
+        h_views[k].copy_(t)
+    dev = [packed_buffers(host_src, device, False) for _ in range(2)]
+    outs = [torch.empty_like(gs.out) for _ in range(2)]
+    out_host = [torch.empty(gs.out.shape, dtype=gs.out.dtype).pin_memory() for _ in range(2)]
+    h2d = h_raw.numel()
+    d2h = out_host[0].numel() * out_host[0].element_size()
+    comp = gs.stream
+    up = torch.cuda.Stream(device)
+    down = torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()
+    uploaded = [ev(), ev()]
+    computed = [ev(), ev()]
+    downloaded = [ev(), ev()]
+    for e in computed + downloaded:
+        e.record(comp)
 
     def one(i):
-        for k, t in host.items():
-            dev_bufs[k].copy_(t, non_blocking=True)
-        gs.run(i)
-        out_host.copy_(gs.out, non_blocking=True)
+        k = i & 1
+        up.wait_event(computed[k])                  # step i-2 no longer reads this set
+        with torch.cuda.stream(up):
+            dev[k][0].copy_(h_raw, non_blocking=True)
+        uploaded[k].record(up)
+        comp.wait_event(uploaded[k])
+        comp.wait_event(downloaded[k])              # step i-2's output has left
+        bufs = dict(dev[k][1])
+        bufs["out"] = outs[k]
+        gs.run(i, bufs=bufs)
+        computed[k].record(comp)
+        down.wait_event(computed[k])
+        with torch.cuda.stream(down):
+            out_host[k].copy_(outs[k], non_blocking=True)
+        downloaded[k].record(down)
 
-    for i in range(3):
+    for i in range(4):
         one(i)
     torch.cuda.synchronize(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(s)
+    e0.record(comp)
+    up.wait_event(e0)
     for i in range(steps):
         one(i)
-    e1.record(s)
+    comp.wait_event(downloaded[(steps - 1) & 1])     # the last output is on the host
+    e1.record(comp)
     e1.synchronize()
+    torch.cuda.synchronize(device)
+    # same inputs as the resident run and a deterministic schedule: same bits
+    if not torch.equal(out_host[(steps - 1) & 1], gs.out.cpu()):
+        raise SystemExit("end-to-end output differs from the resident run's")
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
