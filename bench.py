@@ -161,6 +161,24 @@ def pci_bus_id(dev):
     return None
 
 
+def gpu_local_cpus(bus):
+    """CPUs on the GPU's own NUMA node (sysfs ``local_cpulist``), or None."""
+    if not bus:
+        return None
+    dom, rest = bus.lower().split(":", 1)
+    path = f"/sys/bus/pci/devices/{dom[-4:]}:{rest}/local_cpulist"
+    try:
+        text = open(path).read().strip()
+    except OSError:
+        return None
+    cpus = set()
+    for part in text.split(","):
+        lo, _, hi = part.partition("-")
+        cpus.update(range(int(lo), int(hi or lo) + 1))
+    cpus &= os.sched_getaffinity(0)
+    return cpus or None
+
+
 def combine_over_ranks(dist, ms, nbytes, nseqs, device):
     """(max device ms, total bytes, total sequences) over all ranks.
 
@@ -266,6 +284,11 @@ def e2e_run(pkv, w, gs, steps, device):
     pairs: one packed pinned buffer, one copy) and reads its attention output
     back to pinned host memory.  Two buffer sets alternate, so step i+1's
     upload and step i-1's download run on copy streams while step i computes."""
+    # host threads and pinned buffers on the GPU's NUMA node: copies then
+    # cross no socket link
+    local = gpu_local_cpus(pci_bus_id(device.index if device.index is not None else 0))
+    if local:
+        os.sched_setaffinity(0, local)
     host_src = dict(q=w.q.cpu(), k_new=w.k_new.cpu(), v_new=w.v_new.cpu(),
                     tables=torch.from_numpy(w.block_tables), lens=torch.from_numpy(w.seq_lens),
                     slots=torch.from_numpy(w.slot_mapping), pairs=torch.from_numpy(w.copy_pairs))
@@ -320,7 +343,7 @@ def e2e_run(pkv, w, gs, steps, device):
     # same inputs as the resident run and a deterministic schedule: same bits
     if not torch.equal(out_host[(steps - 1) & 1], gs.out.cpu()):
         raise SystemExit("end-to-end output differs from the resident run's")
-    return e0.elapsed_time(e1) / steps, h2d, d2h
+    return e0.elapsed_time(e1) / steps, h2d, d2h, (len(local) if local else None)
 
 
 # ---------------------------------------------------------------------------
@@ -557,11 +580,13 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e_ms, h2d, d2h = e2e_run(pkv, w, gs, args.e2e_steps, device)
+        e_ms, h2d, d2h, ncpu = e2e_run(pkv, w, gs, args.e2e_steps, device)
         e_ms = combine_over_ranks(dist, e_ms, 0, 0, device)[0]
         e2e = {"value": bytes_total / (e_ms * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": e_ms, "steps": args.e2e_steps}
+               "ms_per_step": e_ms, "steps": args.e2e_steps,
+               "pipeline": "double-buffered: upload of step i+1 and download of step i-1 on copy streams while step i computes",
+               "host_cpus": f"{ncpu} GPU-local CPUs" if ncpu else "affinity unchanged"}
 
     peak, peak_kind = load_peak()
     q_out_bytes = 2 * w.num_seqs * spec.num_q_heads * spec.head_dim * 2

@@ -201,14 +201,18 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
     int* s_prefix = reinterpret_cast<int*>(smem + C::PREFIX_OFF);
 
     // ---- plan: prefix of tiles per sequence, T, the schedule -------------------------
+    // For up to PREFIX_SMEM / 2 - 1 sequences the clamped lengths are kept in
+    // the upper half of the prefix array, so no later length read leaves the SM.
+    const bool lens_smem = N < PREFIX_SMEM / 2;
+    int* s_len = s_prefix + PREFIX_SMEM / 2;
     long long T = 0;
-    for (int base = 0; base < N; base += NT) {
+    auto scan_chunk = [&](int base, int raw) {
         const int s = base + tid;
         long long v = 0;
         if (s < N) {
-            const int raw = __ldg(a.seq_lens + s);
             const int len = clamp_len(raw, cap);
             v = (long long)Hkv * ((len + TILE - 1) / TILE);
+            if (lens_smem) s_len[s] = len;
             if (blockIdx.x == 0) {
                 if (raw > cap) raise_status(PKV_DEV_LENGTH);
                 if (len == 0) {   // nothing to attend to: zero output
@@ -224,6 +228,24 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
             else a.prefix_g[s + 1] = incl;     // every CTA writes the same values
         }
         T += tot;
+    };
+    if (pre_smem) {
+        // every length this thread scans, loaded before the first scan: one round trip
+        constexpr int MAXC = (PREFIX_SMEM + NT - 1) / NT;
+        int raw[MAXC];
+#pragma unroll
+        for (int c = 0; c < MAXC; ++c) {
+            const int s = c * NT + tid;
+            raw[c] = s < N ? __ldg(a.seq_lens + s) : 0;
+        }
+#pragma unroll
+        for (int c = 0; c < MAXC; ++c)
+            if (c * NT < N) scan_chunk(c * NT, raw[c]);
+    } else {
+        for (int base = 0; base < N; base += NT) {
+            const int s = base + tid;
+            scan_chunk(base, s < N ? __ldg(a.seq_lens + s) : 0);
+        }
     }
     if (tid == 0) {
         if (pre_smem) s_prefix[0] = 0;
@@ -279,7 +301,10 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int lb = base + lane;
         return (lb * BS < len) ? __ldg(a.block_tables + (size_t)s * a.max_blocks + lb) : -1;
     };
-    auto seq_len = [&](int s) -> int { return s < N ? clamp_len(__ldg(a.seq_lens + s), cap) : 0; };
+    auto seq_len = [&](int s) -> int {
+        if (s >= N) return 0;
+        return lens_smem ? s_len[s] : clamp_len(__ldg(a.seq_lens + s), cap);
+    };
     auto advance_unit = [&]() {
         pt = 0;
         if (++ph < Hkv) return;
@@ -412,76 +437,111 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         const long long nt = (m.len + TILE - 1) / TILE;
         const long long au = m.f - m.t;                    // the unit's first flat tile
-        const long long bu = au + nt;
-        const int slot = (au < sc.begin(m.r)) ? 0 : 1;     // 0: the unit began in an earlier range
-        const size_t pbase = ((size_t)m.r * 2 + slot) * G;
-        if (g_row < G) {
-            float* po = a.part_o + (pbase + g_row) * D + 2 * c4;
-#pragma unroll
-            for (int n = 0; n < D / 8; ++n)
-                st_cg(reinterpret_cast<float2*>(po + 8 * n), make_float2(ws.o[n][0], ws.o[n][1]));
-            if (c4 == 0) st_cg(a.part_mz + pbase + g_row, make_float2(ws.m, l));
-        }
-        __threadfence();
-        __syncwarp();
         const long long r_lo = sc.range_of(au);
-        const long long r_hi = sc.range_of(bu - 1);
-        unsigned prev = 0;
-        if (lane == 0) prev = atomicAdd(a.tickets + unit, 1u);
-        prev = __shfl_sync(FULL, prev, 0);
-        if (prev != (unsigned)(r_hi - r_lo)) return;      // not the last piece
-        __threadfence();
-        if (lane == 0) st_cg(reinterpret_cast<int*>(a.tickets) + unit, 0);   // ready for the next launch
-        // merge every piece of this unit (max-rescaled), in range order
-        float M[G], den[G];
+        const long long r_hi = sc.range_of(au + nt - 1);
+        const unsigned others = (unsigned)(r_hi - r_lo);   // pieces in other ranges
+        // partial slot of range j: 0 if the unit began in an earlier range
+        auto piece_row = [&](long long j) -> size_t {
+            return ((size_t)j * 2 + ((au < sc.begin(j)) ? 0 : 1)) * G + g_row;
+        };
+        auto store_mine = [&]() {
+            if (g_row < G) {
+                const size_t pr = piece_row(m.r);
+                float* po = a.part_o + pr * D + 2 * c4;
 #pragma unroll
-        for (int g = 0; g < G; ++g) { M[g] = -INFINITY; den[g] = 0.f; }
-        for (long long j = r_lo; j <= r_hi; ++j) {
-            const int sl = (au < sc.begin(j)) ? 0 : 1;
-#pragma unroll
-            for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], ld_cg(a.part_mz + ((size_t)j * 2 + sl) * G + g).x);
-        }
-        constexpr int V4 = G * D / 4;                       // float4 per piece
-        constexpr int PER = (V4 + 31) / 32;
-        float4 acc4[PER];
-#pragma unroll
-        for (int i = 0; i < PER; ++i) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-        for (long long j = r_lo; j <= r_hi; ++j) {
-            const int sl = (au < sc.begin(j)) ? 0 : 1;
-            const size_t jb = ((size_t)j * 2 + sl) * G;
-            float cf[G];
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float2 mz = ld_cg(a.part_mz + jb + g);
-                cf[g] = fast_exp2(mz.x - M[g]);
-                den[g] = fmaf(cf[g], mz.y, den[g]);
+                for (int n = 0; n < D / 8; ++n)
+                    st_cg(reinterpret_cast<float2*>(po + 8 * n), make_float2(ws.o[n][0], ws.o[n][1]));
+                if (c4 == 0) st_cg(a.part_mz + pr, make_float2(ws.m, l));
             }
-            const float4* po = reinterpret_cast<const float4*>(a.part_o + jb * D);
+        };
+        // Every other piece already counted on the ticket: this piece is the
+        // last and merges without publishing itself.  Otherwise publish, count,
+        // and merge only if the count makes this piece the last.
+        unsigned seen = 0;
+        if (lane == 0) seen = ld_acquire(a.tickets + unit);
+        seen = __shfl_sync(FULL, seen, 0);
+        bool mine_in_memory = false;
+        if (seen != others) {
+            store_mine();
+            __threadfence();
+            __syncwarp();
+            unsigned prev = 0;
+            if (lane == 0) prev = atomicAdd(a.tickets + unit, 1u);
+            prev = __shfl_sync(FULL, prev, 0);
+            if (prev != others) return;                   // not the last piece
+            __threadfence();
+            mine_in_memory = true;
+        }
+        if (lane == 0) st_cg(reinterpret_cast<int*>(a.tickets) + unit, 0);   // ready for the next launch
+        // Fold the pieces in range order into this lane's row of the register
+        // state: (M, Z, o) <- (M', e^{M-M'} Z + e^{m_j-M'} Z_j, e^{M-M'} o + e^{m_j-M'} o_j),
+        // M' = max(M, m_j).  The order is fixed, so the result does not depend
+        // on which piece merges.  When this piece is not the first, it goes to
+        // memory and the fold starts from the first piece.
+        float M = ws.m, Z = l;
+        long long j0 = r_lo + 1;
+        if (m.r != r_lo) {
+            if (!mine_in_memory) store_mine();
+            __syncwarp();
+            if (g_row < G) {
+                const size_t pr = piece_row(r_lo);
+                const float* po = a.part_o + pr * D + 2 * c4;
 #pragma unroll
-            for (int i = 0; i < PER; ++i) {
-                const int e = lane + 32 * i;
-                if (e < V4) {
-                    const float4 v = ld_cg(po + e);
-                    const float cg = pick<G>(cf, (e * 4) / D);
-                    acc4[i].x = fmaf(cg, v.x, acc4[i].x);
-                    acc4[i].y = fmaf(cg, v.y, acc4[i].y);
-                    acc4[i].z = fmaf(cg, v.z, acc4[i].z);
-                    acc4[i].w = fmaf(cg, v.w, acc4[i].w);
+                for (int n = 0; n < D / 8; ++n) {
+                    const float2 v = ld_cg(reinterpret_cast<const float2*>(po + 8 * n));
+                    ws.o[n][0] = v.x;
+                    ws.o[n][1] = v.y;
+                }
+                const float2 mz = ld_cg(a.part_mz + pr);
+                M = mz.x;
+                Z = mz.y;
+            }
+        }
+        // head_dim 64: the next piece's loads are issued before this one is
+        // folded in; head_dim 128 has no registers to spare for that
+        constexpr bool PREFETCH = D == 64;
+        float2 v[D / 8], mz = make_float2(0.f, 0.f);
+        auto fetch = [&](long long j) {
+            if (g_row < G) {
+                const size_t pr = piece_row(j);
+                const float* po = a.part_o + pr * D + 2 * c4;
+#pragma unroll
+                for (int n = 0; n < D / 8; ++n) v[n] = ld_cg(reinterpret_cast<const float2*>(po + 8 * n));
+                mz = ld_cg(a.part_mz + pr);
+            }
+        };
+        if (PREFETCH && j0 <= r_hi) fetch(j0);
+        for (long long j = j0; j <= r_hi; ++j) {
+            float2 w[D / 8], wz;
+            if (PREFETCH) {
+#pragma unroll
+                for (int n = 0; n < D / 8; ++n) w[n] = v[n];
+                wz = mz;
+                if (j < r_hi) fetch(j + 1);
+            } else {
+                fetch(j);
+#pragma unroll
+                for (int n = 0; n < D / 8; ++n) w[n] = v[n];
+                wz = mz;
+            }
+            if (g_row < G) {
+                const float mx = fmaxf(M, wz.x);
+                const float ca = fast_exp2(M - mx), cb = fast_exp2(wz.x - mx);
+                Z = fmaf(cb, wz.y, Z * ca);
+                M = mx;
+#pragma unroll
+                for (int n = 0; n < D / 8; ++n) {
+                    ws.o[n][0] = fmaf(cb, w[n].x, ws.o[n][0] * ca);
+                    ws.o[n][1] = fmaf(cb, w[n].y, ws.o[n][1] * ca);
                 }
             }
         }
-        uint16_t* o = a.out + ((size_t)m.s * Hq + (size_t)m.h * G) * D;
+        if (g_row < G) {
+            const float inv = 1.0f / Z;
 #pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            const int e = lane + 32 * i;
-            if (e < V4) {
-                const float inv = 1.0f / pick<G>(den, (e * 4) / D);
-                uint2 pk;
-                pk.x = pack_bf16x2(acc4[i].x * inv, acc4[i].y * inv);
-                pk.y = pack_bf16x2(acc4[i].z * inv, acc4[i].w * inv);
-                *reinterpret_cast<uint2*>(o + (size_t)e * 4) = pk;
-            }
+            for (int n = 0; n < D / 8; ++n)
+                *reinterpret_cast<uint32_t*>(out_row + 8 * n) =
+                    pack_bf16x2(ws.o[n][0] * inv, ws.o[n][1] * inv);
         }
     };
 

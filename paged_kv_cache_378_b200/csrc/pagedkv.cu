@@ -109,31 +109,17 @@ constexpr int attn_stages() {
                : PKV_ATTN_STAGE_BUDGET / (2 * pkv::TileSmem<D, BS>::KT_BYTES);
 }
 
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
 struct WorkspaceLayout {
     size_t prefix_off, mz_off, o_off, tickets_off, total;
     int R_max;
     int cap_tiles;
 };
 
-size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
-// The tile prefix of large batches, two partials per range (one warp of the
-// largest grid this device can run is one range; a cap adds one range per
-// cap-length piece of the longest possible batch), one ticket per
-// (sequence, kv head).
-bool workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                      int max_blocks, int block_size, int partition_tokens, WorkspaceLayout* w) {
-    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
-        !supported_head_dim(head_dim) || max_blocks <= 0 || !supported_block_size(block_size))
-        return false;
-    const int pt = resolve_partition(head_dim, block_size, partition_tokens);
-    if (pt < 0) return false;
-    const int tile = tile_tokens(head_dim, block_size);
-    const long long max_tiles = ((long long)max_blocks * block_size + tile - 1) / tile;
-    long long r_max = (long long)device_sm_count() * kMaxCtasPerSm * kAttnWarps;
-    const int cap_tiles = pt / tile;
-    if (cap_tiles > 0)
-        r_max += ((long long)num_seqs * num_kv_heads * max_tiles + cap_tiles - 1) / cap_tiles + 1;
+// Regions of a workspace holding r_max ranges.
+bool fill_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, long long r_max,
+                 int cap_tiles, WorkspaceLayout* w) {
     if (r_max > (1LL << 30)) return false;
     const size_t G = (size_t)(num_q_heads / num_kv_heads);
     const size_t N = (size_t)num_seqs;
@@ -145,6 +131,28 @@ bool workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_
     w->tickets_off = w->o_off + align_up((size_t)r_max * 2 * G * head_dim * sizeof(float), 256);
     w->total = w->tickets_off + align_up(N * num_kv_heads * sizeof(unsigned int), 256);
     return true;
+}
+
+int grid_warps_for(int D, int G, int BS);
+
+// The tile prefix of large batches, two partials per range (one range per
+// warp of the grid this instance runs on this device; a cap adds one range
+// per cap-length piece of the longest possible batch), one ticket per
+// (sequence, kv head).
+bool workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                      int max_blocks, int block_size, int partition_tokens, WorkspaceLayout* w) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
+        !supported_head_dim(head_dim) || max_blocks <= 0 || !supported_block_size(block_size))
+        return false;
+    const int pt = resolve_partition(head_dim, block_size, partition_tokens);
+    if (pt < 0) return false;
+    const int tile = tile_tokens(head_dim, block_size);
+    const long long max_tiles = ((long long)max_blocks * block_size + tile - 1) / tile;
+    long long r_max = grid_warps_for(head_dim, num_q_heads / num_kv_heads, block_size);
+    const int cap_tiles = pt / tile;
+    if (cap_tiles > 0)
+        r_max += ((long long)num_seqs * num_kv_heads * max_tiles + cap_tiles - 1) / cap_tiles + 1;
+    return fill_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, r_max, cap_tiles, w);
 }
 
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime
@@ -267,21 +275,11 @@ bool noalloc_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
     if (pt < 0) return false;
     const int tile = tile_tokens(head_dim, block_size);
     const long long max_tiles = ((long long)max_blocks * block_size + tile - 1) / tile;
-    long long r_max = grid_warps;
+    long long r_cap = 0;
     const int cap_tiles = pt / tile;
     if (cap_tiles > 0)
-        r_max += ((long long)num_seqs * num_kv_heads * max_tiles + cap_tiles - 1) / cap_tiles + 1;
-    if (r_max > (1LL << 30)) return false;
-    const size_t G = (size_t)(num_q_heads / num_kv_heads);
-    const size_t N = (size_t)num_seqs;
-    w->R_max = (int)r_max;
-    w->cap_tiles = cap_tiles;
-    w->prefix_off = 0;
-    w->mz_off = N > (size_t)pkv::PREFIX_SMEM ? align_up((N + 1) * sizeof(long long), 256) : 0;
-    w->o_off = w->mz_off + align_up((size_t)r_max * 2 * G * sizeof(float2), 256);
-    w->tickets_off = w->o_off + align_up((size_t)r_max * 2 * G * head_dim * sizeof(float), 256);
-    w->total = w->tickets_off + align_up(N * num_kv_heads * sizeof(unsigned int), 256);
-    return true;
+        r_cap = ((long long)num_seqs * num_kv_heads * max_tiles + cap_tiles - 1) / cap_tiles + 1;
+    return fill_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, grid_warps + r_cap, cap_tiles, w);
 }
 
 // Device address of the scratch on the current device (set up on first use).
@@ -468,8 +466,8 @@ int pkv_paged_decode_attention_noalloc(const pkv_cache_t* cache, int layer, cons
     if (!ws) return PKV_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
     // the tickets must start at zero; the scratch keeps whatever the last call left
-    const size_t ticket_bytes = (size_t)num_seqs * cache->num_kv_heads * sizeof(unsigned int);
-    if (cudaMemsetAsync(ws + w.tickets_off, 0, ticket_bytes, s) != cudaSuccess) return PKV_ERR_CUDA;
+    if (cudaMemsetAsync(ws + w.tickets_off, 0, w.total - w.tickets_off, s) != cudaSuccess)
+        return PKV_ERR_CUDA;
 
     CUtensorMap mk, mv;
     if (!encode_pool_map(&mk, cache->k_pool, cache) || !encode_pool_map(&mv, cache->v_pool, cache))

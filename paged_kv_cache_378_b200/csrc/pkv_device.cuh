@@ -107,6 +107,13 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 // (.cg: cached in L2 only; volatile asm with a memory clobber, so the compiler
 // keeps them in program order with the atomics and fences around them)
 
+// acquire load at gpu scope: writes made before a release (or a fence and a
+// write) that produced the value read are visible afterwards
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 __device__ __forceinline__ int ld_cg(const int* p) {
     int v;
     asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

@@ -206,7 +206,6 @@ def test_workspace_reuse_is_stable():
     for _ in range(3):
         b = gpu_step(pkv, w, dev, workspace=ws)[0]
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
-    # every split-K counter is back at zero
     # every ticket (the workspace's last 256 bytes here: 64 of them) is back at zero
     assert w.num_seqs * spec.num_kv_heads * 4 == 256
     assert int(ws[-256:].view(torch.int32).abs().sum()) == 0
