@@ -205,7 +205,7 @@ class GpuStep:
     device time of a step.
     """
 
-    def __init__(self, pkv, w, replicas, partition, device):
+    def __init__(self, pkv, w, replicas, partition, device, fused=True):
         from paged_kv_cache_378_b200._lib import PkvCache
         self.lib = pkv.library()
         spec = w.spec
@@ -237,7 +237,8 @@ class GpuStep:
                                      device=device)
         self.scale = ctypes.c_float(spec.scale)
         self.maxb = w.max_blocks
-        self.launches_per_step = (1 if self.npairs else 0) + 2 * self.L
+        self.fused = fused
+        self.launches_per_step = (1 if self.npairs else 0) + (1 if fused else 2) * self.L
 
     def run(self, step_index, evl=None, bufs=None):
         """Launch one step; ``evl`` = per-layer (start, end) events around
@@ -250,15 +251,24 @@ class GpuStep:
         if self.npairs:
             rc |= lib.pkv_block_copy(cref, b["pairs"].data_ptr(), self.npairs, self.sp)
         for layer in range(self.L):
-            rc |= lib.pkv_kv_append(cref, layer, b["k_new"][layer].data_ptr(),
-                                    b["v_new"][layer].data_ptr(), b["slots"].data_ptr(), self.N,
-                                    self.sp)
-            if evl is not None:
-                evl[layer][0].record(self.stream)
-            rc |= lib.pkv_paged_decode_attention(
-                cref, layer, b["q"][layer].data_ptr(), self.N, self.Hq, b["tables"].data_ptr(),
-                self.maxb, b["lens"].data_ptr(), self.scale, b["out"][layer].data_ptr(),
-                self.ws.data_ptr(), self.ws.numel(), self.partition, self.sp)
+            if self.fused:                   # append of the new token fused into attention
+                if evl is not None:
+                    evl[layer][0].record(self.stream)
+                rc |= lib.pkv_append_paged_decode_attention(
+                    cref, layer, b["k_new"][layer].data_ptr(), b["v_new"][layer].data_ptr(),
+                    b["q"][layer].data_ptr(), self.N, self.Hq, b["tables"].data_ptr(), self.maxb,
+                    b["lens"].data_ptr(), self.scale, b["out"][layer].data_ptr(),
+                    self.ws.data_ptr(), self.ws.numel(), self.partition, self.sp)
+            else:
+                rc |= lib.pkv_kv_append(cref, layer, b["k_new"][layer].data_ptr(),
+                                        b["v_new"][layer].data_ptr(), b["slots"].data_ptr(),
+                                        self.N, self.sp)
+                if evl is not None:
+                    evl[layer][0].record(self.stream)
+                rc |= lib.pkv_paged_decode_attention(
+                    cref, layer, b["q"][layer].data_ptr(), self.N, self.Hq, b["tables"].data_ptr(),
+                    self.maxb, b["lens"].data_ptr(), self.scale, b["out"][layer].data_ptr(),
+                    self.ws.data_ptr(), self.ws.numel(), self.partition, self.sp)
             if evl is not None:
                 evl[layer][1].record(self.stream)
         if rc:
@@ -478,6 +488,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--soak-seconds", type=float, default=1.5)
+    ap.add_argument("--two-call", action="store_true",
+                    help="kv_append and attention as two launches per layer (default: one fused launch)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -520,7 +532,7 @@ def main():
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     nrep = max(1, min(16, math.ceil(4 * l2 / pool_bytes)))
     replicas = [(w.k_pool, w.v_pool)] + [(w.k_pool.clone(), w.v_pool.clone()) for _ in range(nrep - 1)]
-    gs = GpuStep(pkv, w, replicas, part, device)
+    gs = GpuStep(pkv, w, replicas, part, device, fused=not args.two_call)
     pkv.get_device_status(reset=True)
 
     # warm-up
@@ -591,7 +603,9 @@ def main():
     peak, peak_kind = load_peak()
     q_out_bytes = 2 * w.num_seqs * spec.num_q_heads * spec.head_dim * 2
     meta_bytes = w.block_tables.nbytes + w.seq_lens.nbytes
-    alg_bytes = unique_bytes + q_out_bytes + meta_bytes
+    # the fused kernel also reads k_new/v_new and stores them in their slots
+    append_bytes = 2 * (2 * w.num_seqs * spec.num_kv_heads * spec.head_dim * 2) if gs.fused else 0
+    alg_bytes = unique_bytes + q_out_bytes + meta_bytes + append_bytes
     achieved = alg_bytes / (attn_avg_ms * 1e-3) / 1e9
     traffic = load_traffic(args.workload, B)
     line = {
@@ -605,7 +619,10 @@ def main():
                                                             spec.head_dim, w.max_blocks, B, part),
                    "l2": f"inputs larger than L2: {nrep} rotating copies of the KV pools, "
                          f"{nrep * pool_bytes / 1e9:.2f} GB vs {l2 / 1e6:.0f} MB L2",
-                   "parallelism": f"dp{world} (independent batches, no collective)"},
+                   "parallelism": f"dp{world} (independent batches, no collective)",
+                   "step": ("block_copy, then per layer one fused append+attention launch"
+                            if gs.fused else
+                            "block_copy, then per layer kv_append and attention launches")},
         "pct_hbm_peak": 100.0 * value / peak,
         "decode_tokens_per_s_per_layer": seqs_total / (ms_per_step * 1e-3),
         "kv_bytes_per_step": {"unique": unique_bytes * spec.num_layers,

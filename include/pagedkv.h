@@ -22,6 +22,15 @@
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Calls return before the GPU work finishes; nothing inside a
  *    call synchronises the host.
+ *  - Kernels are launched with programmatic stream serialization: each one
+ *    may start while the kernel before it on the stream finishes, and waits
+ *    for that kernel to complete before it reads or writes the pools, q,
+ *    k_new, v_new, the tables, the workspace or out.  The one exception:
+ *    the attention kernel reads seq_lens before that wait, so seq_lens
+ *    must be written by copies or kernels that do not release their
+ *    dependents early (cudaTriggerProgrammaticLaunchCompletion): such a
+ *    writer could still be running when the attention kernel starts.  No
+ *    kernel of this library writes seq_lens.
  *  - Return value: PKV_OK, or a negative PKV_ERR_* code when an argument
  *    check fails on the host (nothing is launched) or a launch fails.
  *  - Faults found by the kernels themselves (a block id or slot outside the
@@ -159,9 +168,9 @@ int pkv_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
  * them into one contiguous range (ithelp article 10405755, "PagedAttention
  * 的核心想法"; "Infra: PagedAttention", "按 Block 分配").  Score
  * s_i = scale * q . k_i, softmax over every visible token.  The work over all
- * (sequence, kv head) pairs is cut into one range per warp plus small ranges
- * claimed dynamically; a sequence that spans several ranges is computed in
- * pieces, each keeping (max score
+ * (sequence, kv head) pairs is cut into equal ranges of tiles, one per warp
+ * of the grid (more under a partition cap); a sequence that spans several
+ * ranges is computed in pieces, each keeping (max score
  * m_r, Z_r = sum e^{s_i - m_r}, unnormalised output), and the pieces are
  * merged with o = sum_r e^{m_r - M} Z_r o_r / sum_r e^{m_r - M} Z_r,
  * M = max_r m_r ("Infra: PagedAttention", "按 Block 分配", the merge
@@ -195,6 +204,39 @@ int pkv_paged_decode_attention(const pkv_cache_t* cache, int layer,
                                const int32_t* seq_lens, float scale, void* out,
                                void* workspace, size_t workspace_bytes,
                                int partition_tokens, void* stream);
+
+/*
+ * pkv_append_paged_decode_attention -- one decode step of one layer in one
+ * launch: pkv_kv_append of every sequence's newest token followed by
+ * pkv_paged_decode_attention, for the decode case where sequence s appends
+ * exactly one token, at position seq_lens[s] - 1.  The pages ask for the
+ * block-table lookup, the K/V read and the attention math to be organised
+ * together ("Infra: PagedAttention", "按 Block 分配", the paragraph on what a
+ * PagedAttention kernel has to do); this entry goes one step further and
+ * folds the append into the same kernel.
+ *
+ *   k_new, v_new   bf16 [num_seqs][num_kv_heads][head_dim], 16-byte aligned:
+ *                  the newest token of each sequence.  Its slot is the one
+ *                  the table gives for position seq_lens[s] - 1, i.e. block
+ *                  block_tables[s][(seq_lens[s]-1)/B], row (seq_lens[s]-1)%B;
+ *                  sequences with seq_lens[s] == 0 append nothing.
+ *   other arguments as pkv_paged_decode_attention.
+ *
+ * Result: the pools hold exactly what pkv_kv_append with that slot mapping
+ * would store, and out is what pkv_paged_decode_attention computes over the
+ * updated pools.  The attention reads the new token from k_new/v_new, not
+ * back from the pool.  Precondition (as for any decode step): the block
+ * holding the new slot belongs to this sequence alone (copy-on-write done).
+ * Errors: as pkv_paged_decode_attention; PKV_ERR_NULL if k_new or v_new is
+ * NULL, PKV_ERR_ALIGN if either is not 16-byte aligned.
+ */
+int pkv_append_paged_decode_attention(const pkv_cache_t* cache, int layer,
+                                      const void* k_new, const void* v_new,
+                                      const void* q, int num_seqs, int num_q_heads,
+                                      const int32_t* block_tables, int max_blocks_per_seq,
+                                      const int32_t* seq_lens, float scale, void* out,
+                                      void* workspace, size_t workspace_bytes,
+                                      int partition_tokens, void* stream);
 
 /*
  * pkv_paged_decode_attention_noalloc -- pkv_paged_decode_attention for callers

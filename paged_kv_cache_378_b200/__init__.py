@@ -28,6 +28,7 @@ from ._lib import PkvCache
 
 __all__ = [
     "PagedKVError", "kv_append", "block_copy", "paged_decode_attention",
+    "append_paged_decode_attention",
     "attention_workspace_bytes", "partition_tokens", "make_workspace",
     "get_device_status", "library", "DEV_RANGE", "DEV_LENGTH", "DEV_TIMEOUT",
 ]
@@ -184,6 +185,44 @@ def paged_decode_attention(q, k_pool, v_pool, block_tables, seq_lens, block_size
         seq_lens.data_ptr(), float(scale), out.data_ptr(), ws_ptr, ws_bytes, int(partition_tokens),
         _stream(dev, stream))
     _check(rc, "paged_decode_attention")
+    return out
+
+
+def append_paged_decode_attention(k_new, v_new, q, k_pool, v_pool, block_tables, seq_lens,
+                                  block_size, scale, out, layer=0, workspace=None,
+                                  partition_tokens=0, stream=None):
+    """Fused decode step of one layer: store each sequence's newest token
+    (``k_new``/``v_new`` bf16 ``[N, H_kv, d]``, position ``seq_lens[s] - 1``,
+    slot from the block table) and attend over the updated cache; writes
+    ``out``.  Same result as ``kv_append`` with that slot mapping followed by
+    ``paged_decode_attention``."""
+    cache, (L, NB, H, B, D) = _cache(k_pool, v_pool)
+    if int(block_size) != B:
+        raise ValueError(f"block_size {block_size} does not match the pools ({B})")
+    dev = k_pool.device
+    for t, name in ((k_new, "k_new"), (v_new, "v_new"), (q, "q"), (out, "out")):
+        _need(t, name, torch.bfloat16, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    if q.dim() != 3 or q.shape[2] != D:
+        raise ValueError(f"q must be [N, H_q, {D}]")
+    N, Hq, _ = q.shape
+    if k_new.shape != (N, H, D) or v_new.shape != (N, H, D):
+        raise ValueError(f"k_new and v_new must be [N, {H}, {D}]")
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    if block_tables.dim() != 2 or block_tables.shape[0] != N or seq_lens.shape != (N,):
+        raise ValueError("block_tables must be [N, max_blocks] and seq_lens [N]")
+    maxb = block_tables.shape[1]
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8, dev)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+    rc = library().pkv_append_paged_decode_attention(
+        ctypes.byref(cache), int(layer), k_new.data_ptr(), v_new.data_ptr(), q.data_ptr(), N, Hq,
+        block_tables.data_ptr(), maxb, seq_lens.data_ptr(), float(scale), out.data_ptr(), ws_ptr,
+        ws_bytes, int(partition_tokens), _stream(dev, stream))
+    _check(rc, "append_paged_decode_attention")
     return out
 
 

@@ -66,11 +66,17 @@ struct AttnArgs {
     unsigned int* tickets;         // [N*Hkv] zero at rest
     long long* prefix_g;           // [N+1] tile prefix, used when N > PREFIX_SMEM
     int R_max;                     // ranges the workspace holds
+    // fused append (k_new != nullptr): the new token of sequence s, at
+    // position seq_lens[s] - 1, is stored in its slot and used in place
+    const uint4* k_new;            // [N][Hkv][D] bf16
+    const uint4* v_new;
+    uint16_t* k_pool;              // pool bases (all layers)
+    uint16_t* v_pool;
     int cap_tiles;                 // > 0: no range longer than this many tiles
     int K;                         // warps in the grid
 };
 
-constexpr int PREFIX_SMEM = 1024;      // sequences whose tile prefix fits in shared memory
+constexpr int PREFIX_SMEM = 768;       // sequences whose tile prefix fits in shared memory
 
 // R equal ranges over the flat space of T tiles (R <= T, so none is empty).
 struct Sched {
@@ -95,7 +101,11 @@ struct AttnCfg {
     static constexpr int Q_OFF = RING_BYTES;
     static constexpr int META_OFF = Q_OFF + NW * STAGES * Q_BYTES;
     static constexpr int BAR_OFF = META_OFF + NW * STAGES * META_BYTES;
-    static constexpr int PREFIX_OFF = BAR_OFF + NW * STAGES * 8;
+    // fused append: per stage, the new token's physical block (16-byte
+    // header) and its K and V rows, brought by bulk copies with the tile
+    static constexpr int NEW_BYTES = 16 + 4 * D;
+    static constexpr int NEW_OFF = BAR_OFF + NW * STAGES * 8;
+    static constexpr int PREFIX_OFF = NEW_OFF + NW * STAGES * NEW_BYTES;
     static constexpr int SMEM_BYTES = PREFIX_OFF + (PREFIX_SMEM + 1) * 4 + 1024;   // + alignment slack
     static constexpr int BOX_BYTES = BS * 128;                  // one TMA box: BS rows x 64 dims
     static constexpr int NT = NW * 32;
@@ -181,6 +191,9 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
     unsigned char* qslots = smem + C::Q_OFF + (size_t)warp * STAGES * C::Q_BYTES;
     StageMeta* meta = reinterpret_cast<StageMeta*>(smem + C::META_OFF) + warp * STAGES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF) + warp * STAGES;
+    unsigned char* newrows = smem + C::NEW_OFF + (size_t)warp * STAGES * C::NEW_BYTES;
+    const bool fused_append = a.k_new != nullptr;
+    constexpr int CH = D / 8;                             // 16-byte chunks of a K or V row
 
     if (lane == 0) {
         if (warp == 0) {
@@ -191,7 +204,6 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int st = 0; st < STAGES; ++st) mbar_init(smem_addr(&bars[st]), 1);
         fence_mbar_init();
     }
-    pdl_wait();                                           // earlier kernels' writes are visible
 
     const int N = a.num_seqs;
     const int Hkv = a.num_kv_heads;
@@ -213,13 +225,7 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int len = clamp_len(raw, cap);
             v = (long long)Hkv * ((len + TILE - 1) / TILE);
             if (lens_smem) s_len[s] = len;
-            if (blockIdx.x == 0) {
-                if (raw > cap) raise_status(PKV_DEV_LENGTH);
-                if (len == 0) {   // nothing to attend to: zero output
-                    uint4* o4 = reinterpret_cast<uint4*>(a.out + (size_t)s * Hq * D);
-                    for (int c = 0; c < Hq * D / 8; ++c) o4[c] = make_uint4(0, 0, 0, 0);
-                }
-            }
+            if (blockIdx.x == 0 && raw > cap) raise_status(PKV_DEV_LENGTH);
         }
         long long tot;
         const long long incl = T + block_scan<NT>(v, s_red, &tot) + v;
@@ -250,6 +256,18 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
     if (tid == 0) {
         if (pre_smem) s_prefix[0] = 0;
         else a.prefix_g[0] = 0;
+    }
+    // Planning read only the lengths, which no kernel of this library writes;
+    // from here on the pool and the outputs are touched, so the kernel before
+    // this one on the stream must have finished.
+    pdl_wait();
+    if (blockIdx.x == 0) {                                // nothing to attend to: zero output
+        for (int s = tid; s < N; s += NT) {
+            if (clamp_len(__ldg(a.seq_lens + s), cap) == 0) {
+                uint4* o4 = reinterpret_cast<uint4*>(a.out + (size_t)s * Hq * D);
+                for (int c = 0; c < Hq * D / 8; ++c) o4[c] = make_uint4(0, 0, 0, 0);
+            }
+        }
     }
     const long long K = a.K;
     Sched sc;
@@ -366,14 +384,33 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         int bid[C::BPT];
 #pragma unroll
         for (int j = 0; j < C::BPT; ++j) bid[j] = __shfl_sync(FULL, ids, lb0 - ids_base + j);
+        // physical block of the new token (fused append, unit's last tile)
+        const int nblk = __shfl_sync(FULL, ids, ((plen - 1) / BS - ids_base) & 31);
         if (lane == 0) {
             StageMeta m;
             m.s = ps; m.h = ph; m.t = pt; m.len = plen; m.f = f; m.flags = flags; m.r = (int)r;
             meta[st] = m;
+            if (fused_append && (flags & F_UNIT_END)) {
+                // where the new token's K and V rows go (null: block id out of range)
+                uint16_t* dk = nullptr;
+                uint16_t* dv = nullptr;
+                if (nblk >= 0 && nblk < a.num_blocks) {
+                    const size_t prow =
+                        (size_t)(a.row_base + ((long long)nblk * Hkv + ph) * BS + (plen - 1) % BS);
+                    dk = a.k_pool + prow * D;
+                    dv = a.v_pool + prow * D;
+                }
+                uint16_t** hdr = reinterpret_cast<uint16_t**>(newrows + (size_t)st * C::NEW_BYTES);
+                hdr[0] = dk;
+                hdr[1] = dv;
+            }
             const uint32_t bar = smem_addr(&bars[st]);
             const uint32_t dK = smem_addr(ring + (size_t)st * C::STAGE_BYTES);
             const uint32_t dV = dK + C::KT_BYTES;
             uint32_t bytes = (flags & F_FIRST) ? C::Q_BYTES : 0u;
+            // fused append: the unit's last tile also brings the new token's rows
+            const bool app = fused_append && (flags & F_UNIT_END);
+            if (app) bytes += 4u * D;
             bool bad = false;
 #pragma unroll
             for (int j = 0; j < C::BPT; ++j) {
@@ -387,6 +424,12 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (flags & F_FIRST)
                 bulk_g2s(smem_addr(qslots + (size_t)st * C::Q_BYTES),
                          a.q + ((size_t)ps * Hq + (size_t)ph * G) * D, C::Q_BYTES, bar, pol_stream);
+            if (app) {
+                unsigned char* nb = newrows + (size_t)st * C::NEW_BYTES;
+                const size_t row = ((size_t)ps * Hkv + ph) * CH;       // in 16-byte chunks
+                bulk_g2s(smem_addr(nb + 16), a.k_new + row, 2u * D, bar, pol_stream);
+                bulk_g2s(smem_addr(nb + 16 + 2 * D), a.v_new + row, 2u * D, bar, pol_stream);
+            }
 #pragma unroll
             for (int j = 0; j < C::BPT; ++j) {
                 if (j * BS >= nv || bid[j] < 0 || bid[j] >= a.num_blocks) continue;
@@ -562,6 +605,23 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         unsigned char* sKp = ring + (size_t)st * C::STAGE_BYTES;
         const uint32_t sK = smem_addr(sKp);
         const uint32_t sV = sK + C::KT_BYTES;
+        if (fused_append && (m.flags & F_UNIT_END)) {
+            // Fused append: the unit's last tile holds the new token.  Its rows
+            // came with the stage; they replace the stale row the tile copy
+            // brought and are stored in their slot (one 16-byte chunk a lane).
+            const unsigned char* nb = newrows + (size_t)st * C::NEW_BYTES;
+            if (lane < 2 * CH) {
+                const int c = lane % CH;
+                uint4* dst = reinterpret_cast<uint4* const*>(nb)[lane < CH ? 0 : 1];
+                if (dst) {
+                    const uint4 v = reinterpret_cast<const uint4*>(nb + 16)[lane];   // K row, then V row
+                    *reinterpret_cast<uint4*>(sKp + (lane < CH ? 0 : C::KT_BYTES) +
+                                              TS::offset(m.len - 1 - m.t * TILE, c)) = v;
+                    dst[c] = v;
+                }
+            }
+            __syncwarp();
+        }
         if (m.flags & F_FIRST) {
             load_q_frags<D, G>(qa, reinterpret_cast<const uint16_t*>(qslots + (size_t)st * C::Q_BYTES),
                                lane);

@@ -295,6 +295,69 @@ unsigned char* noalloc_scratch_ptr() {
     return ptrs[dev];
 }
 
+// Shared body of the attention entry points that take a workspace; k_new and
+// v_new non-null = fused append of each sequence's newest token.
+int attention_with_workspace(const pkv_cache_t* cache, int layer, const void* k_new,
+                                    const void* v_new, const void* q, int num_seqs, int num_q_heads,
+                                    const int32_t* block_tables, int max_blocks_per_seq,
+                                    const int32_t* seq_lens, float scale, void* out, void* workspace,
+                                    size_t workspace_bytes, int partition_tokens, void* stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if (layer < 0 || layer >= cache->num_layers) return PKV_ERR_LAYER;
+    if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || partition_tokens < 0)
+        return PKV_ERR_SHAPE;
+    if (num_q_heads % cache->num_kv_heads) return PKV_ERR_SHAPE;
+    if (!std::isfinite(scale)) return PKV_ERR_SHAPE;
+    const int G = num_q_heads / cache->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PKV_OK;
+    if ((long long)max_blocks_per_seq * cache->block_size > (1LL << 30)) return PKV_ERR_SHAPE;
+    if (!q || !block_tables || !seq_lens || !out) return PKV_ERR_NULL;
+    if (!aligned16(q) || !aligned16(out)) return PKV_ERR_ALIGN;
+    if ((k_new == nullptr) != (v_new == nullptr)) return PKV_ERR_NULL;
+    if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return PKV_ERR_ALIGN;
+    const int D = cache->head_dim, BS = cache->block_size;
+    const int grid_warps = grid_warps_for(D, G, BS);
+    WorkspaceLayout w;
+    if (!workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, D, max_blocks_per_seq, BS,
+                          partition_tokens, &w))
+        return PKV_ERR_SHAPE;
+    if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
+    if (grid_warps > w.R_max) return PKV_ERR_WORKSPACE;
+
+    CUtensorMap mk, mv;
+    if (!encode_pool_map(&mk, cache->k_pool, cache) || !encode_pool_map(&mv, cache->v_pool, cache))
+        return PKV_ERR_CUDA;
+    pkv::AttnArgs a;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    a.q = static_cast<const uint16_t*>(q);
+    a.out = static_cast<uint16_t*>(out);
+    a.block_tables = block_tables;
+    a.seq_lens = seq_lens;
+    a.num_seqs = num_seqs;
+    a.num_kv_heads = cache->num_kv_heads;
+    a.num_blocks = cache->num_blocks;
+    a.max_blocks = max_blocks_per_seq;
+    a.qscale = (float)((double)scale * 1.4426950408889634074);   // scale * log2(e)
+    a.row_base = (long long)layer * cache->num_blocks * cache->num_kv_heads * cache->block_size;
+    a.part_mz = reinterpret_cast<float2*>(ws + w.mz_off);
+    a.part_o = reinterpret_cast<float*>(ws + w.o_off);
+    a.tickets = reinterpret_cast<unsigned int*>(ws + w.tickets_off);
+    a.prefix_g = reinterpret_cast<long long*>(ws + w.prefix_off);
+    a.R_max = w.R_max;
+    a.k_new = static_cast<const uint4*>(k_new);
+    a.v_new = static_cast<const uint4*>(v_new);
+    a.k_pool = static_cast<uint16_t*>(cache->k_pool);
+    a.v_pool = static_cast<uint16_t*>(cache->v_pool);
+    a.cap_tiles = w.cap_tiles;
+    a.K = grid_warps;
+    cudaStream_t s = (cudaStream_t)stream;
+    return with_instance(D, G, BS, [&](auto inst) {
+        return decltype(inst)::launch(mk, mv, a, grid_warps / kAttnWarps, s);
+    });
+}
+
 }  // namespace
 
 extern "C" {
@@ -388,54 +451,21 @@ int pkv_paged_decode_attention(const pkv_cache_t* cache, int layer, const void* 
                                int num_q_heads, const int32_t* block_tables, int max_blocks_per_seq,
                                const int32_t* seq_lens, float scale, void* out, void* workspace,
                                size_t workspace_bytes, int partition_tokens, void* stream) {
-    int rc = check_cache(cache);
-    if (rc) return rc;
-    if (layer < 0 || layer >= cache->num_layers) return PKV_ERR_LAYER;
-    if (num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || partition_tokens < 0)
-        return PKV_ERR_SHAPE;
-    if (num_q_heads % cache->num_kv_heads) return PKV_ERR_SHAPE;
-    if (!std::isfinite(scale)) return PKV_ERR_SHAPE;
-    const int G = num_q_heads / cache->num_kv_heads;
-    if (G != 1 && G != 2 && G != 4 && G != 8) return PKV_ERR_UNSUPPORTED;
-    if (num_seqs == 0) return PKV_OK;
-    if ((long long)max_blocks_per_seq * cache->block_size > (1LL << 30)) return PKV_ERR_SHAPE;
-    if (!q || !block_tables || !seq_lens || !out) return PKV_ERR_NULL;
-    if (!aligned16(q) || !aligned16(out)) return PKV_ERR_ALIGN;
-    const int D = cache->head_dim, BS = cache->block_size;
-    const int grid_warps = grid_warps_for(D, G, BS);
-    WorkspaceLayout w;
-    if (!workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, D, max_blocks_per_seq, BS,
-                          partition_tokens, &w))
-        return PKV_ERR_SHAPE;
-    if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
-    if (grid_warps > w.R_max) return PKV_ERR_WORKSPACE;
+    return attention_with_workspace(cache, layer, nullptr, nullptr, q, num_seqs, num_q_heads,
+                                    block_tables, max_blocks_per_seq, seq_lens, scale, out, workspace,
+                                    workspace_bytes, partition_tokens, stream);
+}
 
-    CUtensorMap mk, mv;
-    if (!encode_pool_map(&mk, cache->k_pool, cache) || !encode_pool_map(&mv, cache->v_pool, cache))
-        return PKV_ERR_CUDA;
-    pkv::AttnArgs a;
-    unsigned char* ws = static_cast<unsigned char*>(workspace);
-    a.q = static_cast<const uint16_t*>(q);
-    a.out = static_cast<uint16_t*>(out);
-    a.block_tables = block_tables;
-    a.seq_lens = seq_lens;
-    a.num_seqs = num_seqs;
-    a.num_kv_heads = cache->num_kv_heads;
-    a.num_blocks = cache->num_blocks;
-    a.max_blocks = max_blocks_per_seq;
-    a.qscale = (float)((double)scale * 1.4426950408889634074);   // scale * log2(e)
-    a.row_base = (long long)layer * cache->num_blocks * cache->num_kv_heads * cache->block_size;
-    a.part_mz = reinterpret_cast<float2*>(ws + w.mz_off);
-    a.part_o = reinterpret_cast<float*>(ws + w.o_off);
-    a.tickets = reinterpret_cast<unsigned int*>(ws + w.tickets_off);
-    a.prefix_g = reinterpret_cast<long long*>(ws + w.prefix_off);
-    a.R_max = w.R_max;
-    a.cap_tiles = w.cap_tiles;
-    a.K = grid_warps;
-    cudaStream_t s = (cudaStream_t)stream;
-    return with_instance(D, G, BS, [&](auto inst) {
-        return decltype(inst)::launch(mk, mv, a, grid_warps / kAttnWarps, s);
-    });
+int pkv_append_paged_decode_attention(const pkv_cache_t* cache, int layer, const void* k_new,
+                                      const void* v_new, const void* q, int num_seqs,
+                                      int num_q_heads, const int32_t* block_tables,
+                                      int max_blocks_per_seq, const int32_t* seq_lens, float scale,
+                                      void* out, void* workspace, size_t workspace_bytes,
+                                      int partition_tokens, void* stream) {
+    if (!k_new || !v_new) return PKV_ERR_NULL;
+    return attention_with_workspace(cache, layer, k_new, v_new, q, num_seqs, num_q_heads,
+                                    block_tables, max_blocks_per_seq, seq_lens, scale, out, workspace,
+                                    workspace_bytes, partition_tokens, stream);
 }
 
 int pkv_paged_decode_attention_noalloc(const pkv_cache_t* cache, int layer, const void* q,
@@ -487,6 +517,10 @@ int pkv_paged_decode_attention_noalloc(const pkv_cache_t* cache, int layer, cons
     a.part_o = reinterpret_cast<float*>(ws + w.o_off);
     a.tickets = reinterpret_cast<unsigned int*>(ws + w.tickets_off);
     a.prefix_g = reinterpret_cast<long long*>(ws + w.prefix_off);
+    a.k_new = nullptr;                                // no fused append here
+    a.v_new = nullptr;
+    a.k_pool = static_cast<uint16_t*>(cache->k_pool);
+    a.v_pool = static_cast<uint16_t*>(cache->v_pool);
     a.R_max = w.R_max;
     a.cap_tiles = w.cap_tiles;
     a.K = grid_warps;

@@ -37,8 +37,12 @@ def device_inputs(w, device="cuda"):
     )
 
 
-def gpu_step(pkv, w, dev_in, layers=None, partition_tokens=None, workspace=None):
-    """Run the step with the CUDA library; returns {layer: out bf16 tensor}."""
+def gpu_step(pkv, w, dev_in, layers=None, partition_tokens=None, workspace=None, fused=False):
+    """Run the step with the CUDA library; returns {layer: out bf16 tensor}.
+
+    ``fused``: append and attention of each layer in one call
+    (``append_paged_decode_attention``) instead of ``kv_append`` then
+    ``paged_decode_attention``."""
     spec = w.spec
     part = spec.partition_tokens if partition_tokens is None else partition_tokens
     L = dev_in["k_pool"].shape[0]
@@ -50,9 +54,16 @@ def gpu_step(pkv, w, dev_in, layers=None, partition_tokens=None, workspace=None)
     pkv.block_copy(dev_in["pairs"], dev_in["k_pool"], dev_in["v_pool"])
     outs = {}
     for layer in layers:
+        out = torch.empty_like(dev_in["q"][layer])
+        if fused:
+            pkv.append_paged_decode_attention(
+                dev_in["k_new"][layer], dev_in["v_new"][layer], dev_in["q"][layer],
+                dev_in["k_pool"], dev_in["v_pool"], dev_in["tables"], dev_in["lens"], w.block_size,
+                spec.scale, out, layer=layer, workspace=workspace, partition_tokens=part)
+            outs[layer] = out
+            continue
         pkv.kv_append(dev_in["k_new"][layer], dev_in["v_new"][layer], dev_in["slots"],
                       dev_in["k_pool"], dev_in["v_pool"], layer=layer)
-        out = torch.empty_like(dev_in["q"][layer])
         pkv.paged_decode_attention(dev_in["q"][layer], dev_in["k_pool"], dev_in["v_pool"],
                                    dev_in["tables"], dev_in["lens"], w.block_size, spec.scale, out,
                                    layer=layer, workspace=workspace, partition_tokens=part)

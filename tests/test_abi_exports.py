@@ -85,6 +85,13 @@ def test_host_argument_checks_before_launch():
     need = lib.pkv_attention_workspace_bytes(2, 8, 2, 64, 4096, 16, 512)
     assert need > 0
     assert att(P(c), 0, 16, 2, 8, 16, 4096, 16, 0.125, 16, 256, need - 1, 512, None) == -4
+    # fused append + attention: both new-row pointers required and aligned
+    fa = lib.pkv_append_paged_decode_attention
+    assert fa(P(c), 0, None, 16, 16, 2, 8, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -1
+    assert fa(P(c), 0, 16, None, 16, 2, 8, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -1
+    assert fa(P(c), 0, 24, 16, 16, 2, 8, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -3
+    assert fa(P(c), 0, 16, 16, 16, 2, 6, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -5
+    assert fa(P(c), 0, 16, 16, 16, 0, 8, 16, 4, 16, 0.125, 16, None, 0, 0, None) == 0
 
 
 def test_workspace_and_partition_sizes():
@@ -107,9 +114,9 @@ def test_workspace_and_partition_sizes():
     per_range = 2 * 4 * (2 + 128) * 4
     assert n0 >= 148 * 4 * per_range + units * 4
     assert n1 - n0 >= (units * 2048 // 32) * per_range
-    # more than 1024 sequences: the tile prefix lives in the workspace too
+    # more than 768 sequences: the tile prefix lives in the workspace too
     big = lib.pkv_attention_workspace_bytes(2048, 32, 8, 64, 16, 16, 0)
-    small = lib.pkv_attention_workspace_bytes(1024, 32, 8, 64, 16, 16, 0)
+    small = lib.pkv_attention_workspace_bytes(768, 32, 8, 64, 16, 16, 0)
     assert big - small >= 2049 * 8
     assert lib.pkv_attention_workspace_bytes(8, 30, 8, 128, 2048, 16, 512) == 0
     assert lib.pkv_attention_workspace_bytes(8, 32, 8, 128, 2048, 12, 512) == 0

@@ -1,0 +1,96 @@
+"""GPU parity of the fused decode step (append of each sequence's newest token
+and attention in one launch) against the oracle and against the two-call path.
+
+Bars: pools bit exact against the oracle's kv_append (the new slots start
+NaN-poisoned, so a missed store shows); attention within
+|gpu - oracle| <= 1e-2 + 1e-2 |oracle|, and bit-identical to kv_append
+followed by paged_decode_attention (same tiles, same order of arithmetic).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as oa
+from workload import make_workload
+from workload.configs import WorkloadSpec
+
+from .stepping import assert_close, device_inputs, f64, gpu_step, oracle_pools_after_step, u16
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import paged_kv_cache_378_b200 as pkv
+else:  # collected on CPU-only machines, never run there
+    pkv = None
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    if torch.cuda.is_available():
+        pkv.get_device_status(reset=True)
+    yield
+
+
+def _fused_vs_oracle_and_two_call(w, partition=None, layers=None):
+    dev_f = device_inputs(w)
+    dev_t = device_inputs(w)
+    outs_f = gpu_step(pkv, w, dev_f, layers=layers, partition_tokens=partition, fused=True)
+    outs_t = gpu_step(pkv, w, dev_t, layers=layers, partition_tokens=partition)
+    assert pkv.get_device_status(reset=True) == 0
+    for l, out in outs_f.items():
+        # pools: the fused store equals kv_append's, bit for bit
+        kp, vp = oracle_pools_after_step(w, u16(w.k_pool[l]), u16(w.v_pool[l]), l)
+        assert np.array_equal(u16(dev_f["k_pool"][l]), kp), f"layer {l}: K pool"
+        assert np.array_equal(u16(dev_f["v_pool"][l]), vp), f"layer {l}: V pool"
+        ref = oa.paged_decode_attention(u16(w.q[l]), kp, vp, w.block_tables, w.seq_lens,
+                                        w.block_size, w.spec.scale)
+        assert_close(f64(out), ref, f"{w.spec.key} layer {l}")
+        assert torch.equal(out.view(torch.int16), outs_t[l].view(torch.int16)), f"layer {l}"
+
+
+@pytest.mark.parametrize("key", ["tiny", "llama1b_layer", "continuous_batch"])
+def test_fused_step_matches_oracle(key):
+    _fused_vs_oracle_and_two_call(make_workload(key))
+
+
+@pytest.mark.parametrize("partition", [512, 0])
+def test_fused_long_context(partition):
+    _fused_vs_oracle_and_two_call(make_workload("long_context"), partition=partition)
+
+
+def _custom(D, G, B, N=6, lens="uniform:1,300", seed=0):
+    return WorkloadSpec(key="custom", title="custom", num_layers=2, num_seqs=N,
+                        num_q_heads=2 * G, num_kv_heads=2, head_dim=D, block_size=B, seed=seed,
+                        lengths=lens)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("B", [4, 16, 32])
+def test_fused_shape_sweep(D, G, B):
+    w = make_workload(_custom(D, G, B, seed=300 + D + 10 * G + B))
+    _fused_vs_oracle_and_two_call(w, partition=64)
+
+
+def test_fused_lengths_one_and_block_boundaries():
+    # length 1: the only token is the new one, so the output is v_new exactly
+    # (after the bf16 round trip); lengths at and just past block multiples
+    w = make_workload(_custom(64, 4, 16, N=7, lens="fixed:1,16,17,32,33,1,48", seed=9))
+    _fused_vs_oracle_and_two_call(w, partition=0)
+    dev = device_inputs(w)
+    out = gpu_step(pkv, w, dev, fused=True)[0]
+    G = w.spec.num_q_heads // w.spec.num_kv_heads
+    for s in np.nonzero(w.seq_lens == 1)[0]:
+        want = w.v_new[0, s].repeat_interleave(G, dim=0)
+        assert torch.equal(out[s].cpu().view(torch.int16), want.view(torch.int16))
+
+
+def test_fused_binding_checks_new_row_shapes():
+    w = make_workload("tiny")
+    dev = device_inputs(w)
+    out = torch.empty_like(dev["q"][0])
+    with pytest.raises(ValueError):
+        pkv.append_paged_decode_attention(dev["k_new"][0][:-1], dev["v_new"][0], dev["q"][0],
+                                          dev["k_pool"], dev["v_pool"], dev["tables"], dev["lens"],
+                                          w.block_size, w.spec.scale, out)
