@@ -68,9 +68,9 @@ def load_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def load_traffic(workload_key, block_size):
+def load_traffic(workload_key, block_size, fused):
     """DRAM bytes per attention launch from the committed ncu summary, or None
-    if absent, for another workload, or taken on different kernel source."""
+    if absent, for another workload or step, or taken on different kernel source."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             rec = json.load(f)
@@ -78,6 +78,7 @@ def load_traffic(workload_key, block_size):
         return None
     for r in rec.get("captures", []):
         if r.get("workload") == workload_key and int(r.get("block_size", -1)) == block_size \
+                and bool(r.get("fused", False)) == fused \
                 and r.get("kernel_source_hash") == kernel_source_hash():
             return r.get("dram_bytes_per_launch")
     return None
@@ -607,7 +608,7 @@ def main():
     append_bytes = 2 * (2 * w.num_seqs * spec.num_kv_heads * spec.head_dim * 2) if gs.fused else 0
     alg_bytes = unique_bytes + q_out_bytes + meta_bytes + append_bytes
     achieved = alg_bytes / (attn_avg_ms * 1e-3) / 1e9
-    traffic = load_traffic(args.workload, B)
+    traffic = load_traffic(args.workload, B, gs.fused)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
