@@ -44,7 +44,9 @@ DEFAULT_WORKLOAD = "continuous_batch"
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "attention_traffic.json")
 EVENT_EVERY = 8            # attention events on every 8th timed step
-KERNEL_SOURCES = ["pkv_device.cuh", "attn_common.cuh", "attn_paged.cuh", "pagedkv.cu"]
+# device sources of the attention kernel: a committed DRAM-traffic capture
+# stands only while these are unchanged
+KERNEL_SOURCES = ["pkv_device.cuh", "attn_common.cuh", "attn_paged.cuh"]
 
 
 # ---------------------------------------------------------------------------
@@ -287,6 +289,118 @@ def packed_buffers(like, device, pin):
     views = {k: raw[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
              for (k, t), o in zip(like.items(), offs.values())}
     return raw, views
+
+
+def prestep_state(w):
+    """The block manager's state before this step, from the step's outputs:
+    lengths minus the new token, new tail blocks removed, copied tails mapped
+    back to their sources, counts from the tables, free blocks in the
+    workload's free-list order."""
+    B = w.block_size
+    lens = w.seq_lens.astype(np.int64) - 1
+    tables = w.block_tables.copy()
+    src_of = {int(d): int(s) for s, d in w.copy_pairs}
+    NB = int(w.num_blocks)
+    ref = np.zeros(NB, np.int64)
+    for s in range(w.num_seqs):
+        lb = int(lens[s]) // B
+        if lens[s] % B == 0:
+            tables[s, lb] = -1
+        elif int(tables[s, lb]) in src_of:
+            tables[s, lb] = src_of[int(tables[s, lb])]
+        nblk = -(-int(lens[s]) // B)
+        np.add.at(ref, tables[s, :nblk], 1)
+    order = w.free_order if w.free_order is not None else np.arange(NB)
+    free = np.array([b for b in order if ref[b] == 0], np.int32)
+    ring = np.full(NB, -1, np.int32)
+    ring[:len(free)] = free
+    return dict(block_tables=tables.astype(np.int32), seq_lens=lens.astype(np.int32),
+                refcount=ref.astype(np.int32), free_ring=ring,
+                free_state=np.array([0, len(free)], np.int32))
+
+
+def block_manager_timing(pkv, w, device, iters=100):
+    """Mean device time of one block-manager step on this workload's pre-step
+    state (restored, untimed, before every launch).  A 256 MB memset queued
+    ahead of each timed launch keeps the GPU busy while the host enqueues, so
+    the events see the kernel, not the host's call overhead."""
+    from paged_kv_cache_378_b200._lib import PkvBlockState
+    pristine = {k: torch.from_numpy(v).to(device) for k, v in prestep_state(w).items()}
+    live = {k: v.clone() for k, v in pristine.items()}
+    c = PkvBlockState(live["block_tables"].data_ptr(), live["seq_lens"].data_ptr(),
+                      live["refcount"].data_ptr(), live["free_ring"].data_ptr(),
+                      live["free_state"].data_ptr())
+    N, maxb = live["block_tables"].shape
+    order = None
+    if w.batch_order is not None:        # the workload's writer order
+        order = torch.from_numpy(np.ascontiguousarray(w.batch_order, dtype=np.int32)).to(device)
+    slots = torch.empty(N, dtype=torch.int64, device=device)
+    pairs = torch.empty((N, 2), dtype=torch.int32, device=device)
+    npairs = torch.zeros(1, dtype=torch.int32, device=device)
+    busy = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    lib = pkv.library()
+    stream = torch.cuda.current_stream(device)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    args = (ctypes.byref(c), N, maxb, int(w.num_blocks), int(w.block_size),
+            order.data_ptr() if order is not None else None, slots.data_ptr(), pairs.data_ptr(),
+            npairs.data_ptr(), sp)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(iters)]
+    for i in range(iters + 5):
+        for k in live:
+            live[k].copy_(pristine[k])
+        busy.zero_()
+        if i >= 5:
+            evs[i - 5][0].record(stream)
+        if lib.pkv_block_manager_step(*args):
+            raise SystemExit("block manager step refused its arguments")
+        if i >= 5:
+            evs[i - 5][1].record(stream)
+    torch.cuda.synchronize(device)
+    if pkv.get_device_status(reset=True):
+        raise SystemExit("device status raised by the block manager step")
+    return sum(a.elapsed_time(b) for a, b in evs) / iters * 1e3
+
+
+def swap_timing(pkv, w, device, blocks=1024, iters=10):
+    """Block swap out to / back in from a pinned host pool: GB/s each way, and
+    a plain pinned cudaMemcpy of the same bytes each way for reference."""
+    L, NB, H, B, D = w.k_pool.shape
+    m = min(blocks, NB)
+    hk = torch.empty((L, m, H, B, D), dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    rng = np.random.default_rng(0)
+    dev_ids = rng.choice(NB, m, replace=False).astype(np.int32)
+    out_pairs = torch.from_numpy(np.stack([dev_ids, np.arange(m, dtype=np.int32)], 1)).to(device)
+    in_pairs = torch.from_numpy(np.stack([np.arange(m, dtype=np.int32), dev_ids], 1)).to(device)
+    nbytes = 2 * hk.numel() * hk.element_size()
+    stream = torch.cuda.current_stream(device)
+    ref_h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    ref_d = torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / iters * 1e-3
+
+    t_out = timed(lambda: pkv.swap_blocks(out_pairs, w.k_pool, w.v_pool, hk, hv, pkv.SWAP_OUT))
+    t_in = timed(lambda: pkv.swap_blocks(in_pairs, w.k_pool, w.v_pool, hk, hv, pkv.SWAP_IN))
+    t_h2d = timed(lambda: ref_d.copy_(ref_h, non_blocking=True))
+    t_d2h = timed(lambda: ref_h.copy_(ref_d, non_blocking=True))
+    if pkv.get_device_status(reset=True):
+        raise SystemExit("device status raised by the block swap")
+    return {"blocks": m, "bytes_each_way": nbytes,
+            "out_gbs": nbytes / t_out / 1e9, "in_gbs": nbytes / t_in / 1e9,
+            "memcpy_d2h_gbs": nbytes / t_d2h / 1e9, "memcpy_h2d_gbs": nbytes / t_h2d / 1e9,
+            "what": "swap of randomly chosen device blocks (all layers, K and V) to a pinned "
+                    "host pool and back, one launch each way; reference: one pinned memcpy of "
+                    "the same bytes"}
 
 
 def e2e_run(pkv, w, gs, steps, device):
@@ -601,6 +715,9 @@ def main():
                "pipeline": "double-buffered: upload of step i+1 and download of step i-1 on copy streams while step i computes",
                "host_cpus": f"{ncpu} GPU-local CPUs" if ncpu else "affinity unchanged"}
 
+    bm_us = block_manager_timing(pkv, w, device) if w.num_seqs <= 4096 else None
+    swap = swap_timing(pkv, w, device)
+
     peak, peak_kind = load_peak()
     q_out_bytes = 2 * w.num_seqs * spec.num_q_heads * spec.head_dim * 2
     meta_bytes = w.block_tables.nbytes + w.seq_lens.nbytes
@@ -636,6 +753,11 @@ def main():
                      "event_sampling": f"attention bracketed on every {EVENT_EVERY}th timed step"},
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "swap": swap,
+        "block_manager": None if bm_us is None else {
+            "us_per_step": bm_us, "num_seqs": w.num_seqs,
+            "what": "device block-manager step (slot mapping, copy-on-write decisions, block "
+                    "allocation) timed alone on this step's pre-step state, restored between launches"},
         "gpu_launches": gs.launches_per_step * args.steps,
         "clocks": clocks,
     }

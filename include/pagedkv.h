@@ -73,6 +73,7 @@ extern "C" {
 #define PKV_ERR_CUDA         -6  /* a CUDA runtime call or launch failed */
 #define PKV_ERR_LAYER        -7  /* layer index outside [0, num_layers) */
 #define PKV_ERR_SCRATCH      -8  /* request too large for the no-allocation scratch */
+#define PKV_ERR_MEMORY       -9  /* a host pool is not pinned (page-locked, mapped) memory */
 
 /* size of the device buffer behind pkv_paged_decode_attention_noalloc */
 #define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -81,6 +82,7 @@ extern "C" {
 #define PKV_DEV_RANGE    0x1u  /* block id or slot outside the pool: access skipped */
 #define PKV_DEV_LENGTH   0x2u  /* seq_len above max_blocks_per_seq * block_size: clamped */
 #define PKV_DEV_TIMEOUT  0x4u  /* a bounded wait for staged KV gave up */
+#define PKV_DEV_NOBLOCKS 0x8u  /* block manager step: not enough free blocks, nothing changed */
 
 typedef struct pkv_cache {
     void*   k_pool;        /* bf16 [num_layers][num_blocks][num_kv_heads][block_size][head_dim] */
@@ -130,6 +132,86 @@ int pkv_kv_append(const pkv_cache_t* cache, int layer,
  */
 int pkv_block_copy(const pkv_cache_t* cache, const int32_t* src_dst_pairs,
                    int num_pairs, void* stream);
+
+/*
+ * pkv_block_copy_device_count -- pkv_block_copy with the pair count read on
+ * the device: copies the first *num_pairs (at most max_pairs) pairs.  For a
+ * step whose copy pairs come from pkv_block_manager_step, so the host never
+ * waits for the count.
+ *
+ *   num_pairs   device int32 [1]
+ *   max_pairs   >= 0, capacity of src_dst_pairs; 0 launches nothing
+ */
+int pkv_block_copy_device_count(const pkv_cache_t* cache, const int32_t* src_dst_pairs,
+                                int max_pairs, const int32_t* num_pairs, void* stream);
+
+/*
+ * pkv_swap_blocks -- move whole blocks between the device pool and a pool in
+ * pinned host memory, every layer, K and V, in one launch.
+ *
+ * Defines: under memory pressure, blocks can be swapped out to CPU memory and
+ * brought back later ("只用了 8 格，為什麼占了 12 格？", 故事沒有說完的部分).
+ *
+ *   device_cache   the device pool (as for the other calls)
+ *   host_cache     a pool of the same layers, kv heads, block size and
+ *                  head_dim in page-locked host memory that the device can
+ *                  address (cudaHostAlloc, or cudaHostRegister with the
+ *                  mapped flag; torch's pin_memory qualifies); its own
+ *                  num_blocks.  Pageable memory gives PKV_ERR_MEMORY.
+ *   src_dst_pairs  device int32 [num_pairs][2]
+ *   direction      PKV_SWAP_OUT: host[l][dst] = device[l][src];
+ *                  PKV_SWAP_IN:  device[l][dst] = host[l][src]
+ * Bit exact.  A block id outside its pool sets PKV_DEV_RANGE and that pair is
+ * skipped.  The copy runs over PCIe inside the kernel (no per-block memcpy).
+ */
+#define PKV_SWAP_OUT 0
+#define PKV_SWAP_IN  1
+int pkv_swap_blocks(const pkv_cache_t* device_cache, const pkv_cache_t* host_cache,
+                    const int32_t* src_dst_pairs, int num_pairs, int direction, void* stream);
+
+/*
+ * Block manager state on the device, for pkv_block_manager_step.  All device
+ * pointers, owned by the caller.
+ */
+typedef struct pkv_block_state {
+    int32_t* block_tables;  /* [num_seqs][max_blocks_per_seq]; entries past a
+                               sequence's blocks are ignored */
+    int32_t* seq_lens;      /* [num_seqs] tokens cached per sequence */
+    int32_t* refcount;      /* [num_blocks] users of each physical block */
+    int32_t* free_ring;     /* [num_blocks] ring of free block ids */
+    int32_t* free_state;    /* [2]: ring index of the next free id, number of free ids */
+} pkv_block_state_t;
+
+/*
+ * pkv_block_manager_step -- one decode step of the block manager, on the
+ * device: every sequence appends one token.
+ *
+ * Defines ("Infra: PagedAttention", "按 Block 分配" and "共享前缀，分叉时
+ * Copy-on-write"; ithelp article 10405755, "手動畫一次 block table"): a new
+ * token fills the tail block; a full tail (or no block) takes the next free
+ * block; a tail with room whose reference count is above one is copied first
+ * (take a free block, record the copy pair, remap, drop one reference on the
+ * old tail).  Writers are served in `order`; each writer that still sees a
+ * count above one copies, so the last of k sharers that all write keeps the
+ * block.  Free blocks are handed out from the ring in order.
+ *
+ *   order          device int32 [num_seqs], a permutation of 0..num_seqs-1
+ *                  (writer order), or NULL for 0..num_seqs-1
+ *   slot_mapping   device int64 [num_seqs] out: slot of each sequence's new
+ *                  token (block * block_size + offset)
+ *   copy_pairs     device int32 [num_seqs][2] out, (src, dst) in writer order
+ *   num_pairs      device int32 [1] out
+ * On return the tables, lengths (+1), counts and free state are updated.
+ * num_seqs <= 4096 (PKV_ERR_UNSUPPORTED above).  If the free blocks do not
+ * suffice, or an order entry, a length or a tail block id is out of range,
+ * the kernel sets PKV_DEV_NOBLOCKS / PKV_DEV_RANGE / PKV_DEV_LENGTH and
+ * changes nothing.  The kernel does not release its dependents early, so an
+ * attention launch that follows on the stream reads the new lengths.
+ */
+int pkv_block_manager_step(const pkv_block_state_t* state, int num_seqs,
+                           int max_blocks_per_seq, int num_blocks, int block_size,
+                           const int32_t* order, int64_t* slot_mapping,
+                           int32_t* copy_pairs, int32_t* num_pairs, void* stream);
 
 /*
  * pkv_attention_workspace_bytes -- bytes of workspace pkv_paged_decode_attention

@@ -87,6 +87,23 @@ def block_copy(k_pools, v_pools, src_dst_pairs):
     return kp, vp
 
 
+def swap_blocks(src_k, src_v, dst_k, dst_v, src_dst_pairs):
+    """Move whole blocks (every layer, every head, K and V) from one pool to
+    another, e.g. device pool -> host pool when memory runs short and back:
+    ``dst[l][d] = src[l][s]`` for each pair (s, d).  [AKIRA] 故事沒有說完的部分:
+    under memory pressure blocks can be swapped out to CPU memory and brought
+    back later.  Returns the new destination pools; the source is unchanged.
+    """
+    sk, sv = _bf16.as_u16(src_k), _bf16.as_u16(src_v)
+    dk = _bf16.as_u16(dst_k).copy()
+    dv = _bf16.as_u16(dst_v).copy()
+    for src, dst in np.asarray(src_dst_pairs).reshape(-1, 2).tolist():
+        for layer in range(dk.shape[0]):
+            dk[layer, dst] = sk[layer, src]
+            dv[layer, dst] = sv[layer, src]
+    return dk, dv
+
+
 # --------------------------------------------------------------------------
 # attention
 # --------------------------------------------------------------------------

@@ -24,18 +24,20 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import PkvCache
+from ._lib import PkvBlockState, PkvCache
 
 __all__ = [
     "PagedKVError", "kv_append", "block_copy", "paged_decode_attention",
-    "append_paged_decode_attention",
+    "append_paged_decode_attention", "BlockState", "block_manager_step", "swap_blocks",
+    "SWAP_OUT", "SWAP_IN",
     "attention_workspace_bytes", "partition_tokens", "make_workspace",
-    "get_device_status", "library", "DEV_RANGE", "DEV_LENGTH", "DEV_TIMEOUT",
+    "get_device_status", "library", "DEV_RANGE", "DEV_LENGTH", "DEV_TIMEOUT", "DEV_NOBLOCKS",
 ]
 
 DEV_RANGE = 0x1
 DEV_LENGTH = 0x2
 DEV_TIMEOUT = 0x4
+DEV_NOBLOCKS = 0x8
 
 
 class PagedKVError(RuntimeError):
@@ -112,10 +114,12 @@ def kv_append(k, v, slot_mapping, k_pool, v_pool, layer=0, stream=None):
     _check(rc, "kv_append")
 
 
-def block_copy(src_dst_pairs, k_pool, v_pool, stream=None):
+def block_copy(src_dst_pairs, k_pool, v_pool, num_pairs=None, stream=None):
     """Copy whole blocks (every layer, K and V): ``pool[:, dst] = pool[:, src]``.
 
-    ``src_dst_pairs``: int32 ``[n, 2]``.
+    ``src_dst_pairs``: int32 ``[n, 2]``.  ``num_pairs``: optional int32 CUDA
+    tensor ``[1]`` holding how many of the ``n`` pairs to copy (read on the
+    device, e.g. the count ``block_manager_step`` wrote).
     """
     cache, _ = _cache(k_pool, v_pool)
     dev = k_pool.device
@@ -123,9 +127,90 @@ def block_copy(src_dst_pairs, k_pool, v_pool, stream=None):
     if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
         raise ValueError("src_dst_pairs must be [n, 2]")
     n = src_dst_pairs.shape[0]
-    rc = library().pkv_block_copy(ctypes.byref(cache), src_dst_pairs.data_ptr(), n,
-                                  _stream(dev, stream))
+    if num_pairs is None:
+        rc = library().pkv_block_copy(ctypes.byref(cache), src_dst_pairs.data_ptr(), n,
+                                      _stream(dev, stream))
+    else:
+        _need(num_pairs, "num_pairs", torch.int32, dev)
+        rc = library().pkv_block_copy_device_count(ctypes.byref(cache), src_dst_pairs.data_ptr(),
+                                                   n, num_pairs.data_ptr(), _stream(dev, stream))
     _check(rc, "block_copy")
+
+
+SWAP_OUT = 0
+SWAP_IN = 1
+
+
+def swap_blocks(src_dst_pairs, k_pool, v_pool, host_k_pool, host_v_pool, direction, stream=None):
+    """Move whole blocks (every layer, K and V) between the device pools and
+    pools in pinned host memory (``tensor.pin_memory()``), same shapes except
+    the block count.  ``direction``: ``SWAP_OUT`` (host[dst] = device[src]) or
+    ``SWAP_IN`` (device[dst] = host[src]); ``src_dst_pairs`` int32 CUDA ``[n, 2]``."""
+    cache, _ = _cache(k_pool, v_pool)
+    for t, name in ((host_k_pool, "host_k_pool"), (host_v_pool, "host_v_pool")):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.is_cuda \
+                or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CPU tensor in pinned memory")
+        if not t.is_pinned():
+            raise ValueError(f"{name} must be pinned (tensor.pin_memory())")
+    if host_k_pool.shape != host_v_pool.shape:
+        raise ValueError("host_k_pool and host_v_pool must have the same shape")
+    L, NB, H, B, D = host_k_pool.shape
+    host = PkvCache(host_k_pool.data_ptr(), host_v_pool.data_ptr(), L, NB, H, B, D)
+    dev = k_pool.device
+    _need(src_dst_pairs, "src_dst_pairs", torch.int32, dev)
+    if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be [n, 2]")
+    rc = library().pkv_swap_blocks(ctypes.byref(cache), ctypes.byref(host), src_dst_pairs.data_ptr(),
+                                   src_dst_pairs.shape[0], int(direction), _stream(dev, stream))
+    _check(rc, "swap_blocks")
+
+
+class BlockState:
+    """Block manager state on the device: tables ``[N, max_blocks]``, lengths
+    ``[N]``, reference counts ``[num_blocks]``, the free ring ``[num_blocks]``
+    and ``free_state = [head, count]`` (all int32 CUDA tensors)."""
+
+    def __init__(self, block_tables, seq_lens, refcount, free_ring, free_state):
+        dev = block_tables.device
+        for t, name in ((block_tables, "block_tables"), (seq_lens, "seq_lens"),
+                        (refcount, "refcount"), (free_ring, "free_ring"),
+                        (free_state, "free_state")):
+            _need(t, name, torch.int32, dev)
+        if block_tables.dim() != 2 or seq_lens.shape != (block_tables.shape[0],):
+            raise ValueError("block_tables must be [N, max_blocks] and seq_lens [N]")
+        if refcount.dim() != 1 or free_ring.shape != refcount.shape or free_state.shape != (2,):
+            raise ValueError("refcount and free_ring must be [num_blocks], free_state [2]")
+        self.block_tables, self.seq_lens = block_tables, seq_lens
+        self.refcount, self.free_ring, self.free_state = refcount, free_ring, free_state
+
+    def _c(self):
+        return PkvBlockState(self.block_tables.data_ptr(), self.seq_lens.data_ptr(),
+                             self.refcount.data_ptr(), self.free_ring.data_ptr(),
+                             self.free_state.data_ptr())
+
+
+def block_manager_step(state, block_size, order=None, stream=None):
+    """One decode step of the block manager on the device (every sequence
+    appends one token; ``order`` int32 ``[N]`` is the writer order).  Updates
+    ``state`` in place; returns ``(slot_mapping int64 [N], copy_pairs int32
+    [N, 2], num_pairs int32 [1])`` on the device."""
+    dev = state.block_tables.device
+    N, maxb = state.block_tables.shape
+    nb = state.refcount.shape[0]
+    if order is not None:
+        _need(order, "order", torch.int32, dev)
+        if order.shape != (N,):
+            raise ValueError("order must be [N]")
+    slots = torch.empty(N, dtype=torch.int64, device=dev)
+    pairs = torch.empty((max(N, 1), 2), dtype=torch.int32, device=dev)
+    npairs = torch.zeros(1, dtype=torch.int32, device=dev)
+    c = state._c()
+    rc = library().pkv_block_manager_step(
+        ctypes.byref(c), N, maxb, nb, int(block_size), order.data_ptr() if order is not None else None,
+        slots.data_ptr(), pairs.data_ptr(), npairs.data_ptr(), _stream(dev, stream))
+    _check(rc, "block_manager_step")
+    return slots, pairs[:N], npairs
 
 
 def attention_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,

@@ -22,12 +22,29 @@ class PkvCache(ctypes.Structure):
     ]
 
 
+class PkvBlockState(ctypes.Structure):
+    _fields_ = [
+        ("block_tables", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p),
+        ("refcount", ctypes.c_void_p),
+        ("free_ring", ctypes.c_void_p),
+        ("free_state", ctypes.c_void_p),
+    ]
+
+
 # name -> (restype, argtypes); mirrors include/pagedkv.h
 SIGNATURES = {
     "pkv_kv_append": (ctypes.c_int, [ctypes.POINTER(PkvCache), ctypes.c_int, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "pkv_block_copy": (ctypes.c_int, [ctypes.POINTER(PkvCache), ctypes.c_void_p, ctypes.c_int,
                                       ctypes.c_void_p]),
+    "pkv_block_copy_device_count": (ctypes.c_int, [ctypes.POINTER(PkvCache), ctypes.c_void_p,
+                                                   ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
+    "pkv_swap_blocks": (ctypes.c_int, [ctypes.POINTER(PkvCache), ctypes.POINTER(PkvCache),
+                                       ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "pkv_block_manager_step": (ctypes.c_int, [
+        ctypes.POINTER(PkvBlockState), ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "pkv_attention_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 7),
     "pkv_partition_tokens": (ctypes.c_int, [ctypes.c_int] * 6),
     "pkv_workspace_init": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),

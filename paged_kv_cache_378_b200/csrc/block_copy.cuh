@@ -13,12 +13,20 @@ namespace pkv {
 // (num_kv_heads * block_size * head_dim bf16 = chunks_per_block 16-byte
 // chunks).  The flattened (unit, chunk) space is walked with a grid stride;
 // four independent chunk copies per thread per step keep loads in flight.
+// Source and destination pools may differ (block swap between the device
+// pool and a pinned host pool): each has its own block count.
 __global__ void __launch_bounds__(256)
-block_copy_kernel(uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
+block_copy_kernel(uint4* __restrict__ dst_k, uint4* __restrict__ dst_v,
+                  const uint4* __restrict__ src_k, const uint4* __restrict__ src_v,
                   const int32_t* __restrict__ pairs, int num_pairs, int num_layers,
-                  int num_blocks, long long chunks_per_block) {
+                  int src_blocks, int dst_blocks, long long chunks_per_block,
+                  const int32_t* __restrict__ d_num_pairs) {   // null: num_pairs is the count
     pdl_launch_dependents();
-    pdl_wait();                                          // earlier writes to the pool land first
+    pdl_wait();                                          // earlier writes to the pools land first
+    if (d_num_pairs) {
+        const int n = *d_num_pairs;
+        num_pairs = n < 0 ? 0 : (n < num_pairs ? n : num_pairs);
+    }
     const long long units = (long long)num_pairs * num_layers * 2;
     const long long total = units * chunks_per_block;
     const long long stride = (long long)gridDim.x * blockDim.x;
@@ -39,14 +47,14 @@ block_copy_kernel(uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
             const int layer = (int)(pl - (long long)pair * num_layers);
             const int src = __ldg(pairs + 2 * pair);
             const int dst = __ldg(pairs + 2 * pair + 1);
-            if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+            if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
                 if (c == 0) raise_status(PKV_DEV_RANGE);
                 continue;
             }
-            uint4* pool = which ? v_pool : k_pool;
-            const size_t layer_base = (size_t)layer * num_blocks * chunks_per_block;
-            v[k] = pool[layer_base + (size_t)src * chunks_per_block + c];
-            dptr[k] = pool + layer_base + (size_t)dst * chunks_per_block + c;
+            const uint4* sp = which ? src_v : src_k;
+            uint4* dp = which ? dst_v : dst_k;
+            v[k] = sp[((size_t)layer * src_blocks + src) * chunks_per_block + c];
+            dptr[k] = dp + ((size_t)layer * dst_blocks + dst) * chunks_per_block + c;
         }
 #pragma unroll
         for (int k = 0; k < 4; ++k)

@@ -1,0 +1,173 @@
+// block_manager_step: one decode step of the block manager on the device.
+//
+// What it computes ("Infra: PagedAttention", sections 按 Block 分配 and 共享前缀，
+// 分叉时 Copy-on-write; ithelp article 10405755, section 手動畫一次 block table):
+// every sequence appends one token.  Writers are served in the given order.
+// A writer whose tail block is full (or who has no block) takes the next free
+// block.  A writer whose tail has room but is shared (reference count above
+// one) copies it: it takes a free block, records (tail, new) as a copy pair,
+// remaps its table and drops one reference on the old tail.  Otherwise it
+// writes in place.  The new token's slot is table[pos / B] * B + pos % B.
+//
+// The order-dependent choices are made without a serial walk:
+//   - a writer on shared tail b sees count c_b - r, where r is the number of
+//     earlier writers on b (each of them copied and dropped one reference),
+//     so it copies exactly when r < c_b - 1;
+//   - the k-th block taken, in writer order, is the free ring's entry at
+//     head + k (an exclusive scan of "takes a block" over the writers);
+//   - copy pairs are numbered by an exclusive scan of "copies".
+// One CTA of 1024 threads; writer i is handled by thread i mod 1024.
+#pragma once
+
+#include "pkv_device.cuh"
+
+namespace pkv {
+
+constexpr int BM_THREADS = 1024;
+constexpr int BM_PER_THREAD = 4;
+constexpr int BM_MAX_SEQS = BM_THREADS * BM_PER_THREAD;
+
+struct BmArgs {
+    int32_t* block_tables;      // [N][max_blocks], updated in place
+    int32_t* seq_lens;          // [N] lengths before the step; + 1 on return
+    int32_t* refcount;          // [num_blocks]
+    const int32_t* free_ring;   // [num_blocks] free block ids, in hand-out order from head
+    int32_t* free_state;        // [2] head (ring index of the next free id), count
+    const int32_t* order;       // [N] writer order (sequence ids), or null: 0..N-1
+    int64_t* slot_mapping;      // [N] out, by sequence
+    int32_t* copy_pairs;        // [N][2] out, (src, dst) in writer order
+    int32_t* num_pairs;         // [1] out
+    int num_seqs;
+    int max_blocks;
+    int num_blocks;
+    int block_size;
+};
+
+// Block-wide exclusive scan of one int per thread (BM_THREADS threads).
+__device__ __forceinline__ int bm_scan(int v, int* s_warp, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = s_warp[lane];                           // BM_THREADS / 32 == 32 warps
+        int incl = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        s_warp[lane] = incl - w;                        // exclusive prefix of warp sums
+        if (lane == 31) s_warp[32] = incl;
+    }
+    __syncthreads();
+    const int before = s_warp[warp] + x - v;
+    *total = s_warp[32];
+    __syncthreads();
+    return before;
+}
+
+__global__ void __launch_bounds__(BM_THREADS, 1) block_manager_kernel(const BmArgs a) {
+    // The tables, lengths and counts may still be read by the kernel before
+    // this one.  This kernel never releases its dependents early: the next
+    // attention launch reads the lengths before its own wait.
+    pdl_wait();
+    __shared__ int s_tail[BM_MAX_SEQS];                 // tail block of writer i, -1: takes a new one
+    __shared__ int s_warp[33];
+    __shared__ int s_abort;
+    const int N = a.num_seqs, B = a.block_size;
+    const int tid = threadIdx.x;
+    if (tid == 0) s_abort = 0;
+
+    // writer i = k * BM_THREADS + tid: one per thread for up to 1024 sequences
+    int seq[BM_PER_THREAD], pos[BM_PER_THREAD], cnt[BM_PER_THREAD];
+#pragma unroll
+    for (int k = 0; k < BM_PER_THREAD; ++k) {
+        const int i = k * BM_THREADS + tid;
+        seq[k] = -1; pos[k] = 0; cnt[k] = 0;
+        if (i >= N) continue;
+        s_tail[i] = -1;
+        const int s = a.order ? a.order[i] : i;
+        if (s < 0 || s >= N) { raise_status(PKV_DEV_RANGE); atomicExch(&s_abort, 1); continue; }
+        seq[k] = s;
+        pos[k] = a.seq_lens[s];
+        const int lb = pos[k] / B;
+        if (pos[k] < 0 || lb >= a.max_blocks) { raise_status(PKV_DEV_LENGTH); atomicExch(&s_abort, 1); continue; }
+        if (pos[k] % B != 0) {
+            const int tail = a.block_tables[(size_t)s * a.max_blocks + lb];
+            if (tail < 0 || tail >= a.num_blocks) { raise_status(PKV_DEV_RANGE); atomicExch(&s_abort, 1); continue; }
+            s_tail[i] = tail;
+            cnt[k] = a.refcount[tail];
+        }
+    }
+    __syncthreads();
+
+    // which writers take a block, which of them copy: only writers on a shared
+    // tail need their rank among earlier writers of the same block
+    int takes[BM_PER_THREAD], copies[BM_PER_THREAD];
+#pragma unroll
+    for (int k = 0; k < BM_PER_THREAD; ++k) {
+        const int i = k * BM_THREADS + tid;
+        takes[k] = copies[k] = 0;
+        if (seq[k] < 0) continue;
+        const int tail = s_tail[i];
+        if (tail < 0) {
+            takes[k] = 1;
+        } else if (cnt[k] > 1) {
+            int r = 0;                                  // earlier writers on the same tail
+            for (int j = 0; j < i && r < cnt[k] - 1; ++j) r += (s_tail[j] == tail);
+            if (cnt[k] - r > 1) takes[k] = copies[k] = 1;
+        }
+    }
+    // exclusive scans in writer order, one round of BM_THREADS writers at a time
+    int take_base[BM_PER_THREAD], copy_base[BM_PER_THREAD];
+    int total_takes = 0, total_copies = 0;
+#pragma unroll
+    for (int k = 0; k < BM_PER_THREAD; ++k) {
+        if (k * BM_THREADS >= N) { take_base[k] = copy_base[k] = 0; continue; }   // uniform
+        int t, c;
+        take_base[k] = total_takes + bm_scan(takes[k], s_warp, &t);
+        copy_base[k] = total_copies + bm_scan(copies[k], s_warp, &c);
+        total_takes += t;
+        total_copies += c;
+    }
+    const int head = a.free_state[0], avail = a.free_state[1];
+    if (s_abort || total_takes > avail) {               // change nothing
+        if (tid == 0 && total_takes > avail) raise_status(PKV_DEV_NOBLOCKS);
+        return;
+    }
+    __syncthreads();                                    // every count read before any is changed
+
+#pragma unroll
+    for (int k = 0; k < BM_PER_THREAD; ++k) {
+        if (seq[k] < 0) continue;
+        const int s = seq[k], p = pos[k];
+        int32_t* entry = a.block_tables + (size_t)s * a.max_blocks + p / B;
+        if (takes[k]) {
+            const int nb = a.free_ring[(head + take_base[k]) % a.num_blocks];
+            if (nb < 0 || nb >= a.num_blocks) { raise_status(PKV_DEV_RANGE); continue; }
+            a.refcount[nb] = 1;
+            if (copies[k]) {
+                const int tail = s_tail[k * BM_THREADS + tid];
+                a.copy_pairs[2 * copy_base[k]] = tail;
+                a.copy_pairs[2 * copy_base[k] + 1] = nb;
+                atomicSub(a.refcount + tail, 1);
+            }
+            *entry = nb;
+        }
+        a.slot_mapping[s] = (int64_t)(*entry) * B + p % B;
+        a.seq_lens[s] = p + 1;
+    }
+    if (tid == 0) {
+        a.free_state[0] = (head + total_takes) % a.num_blocks;
+        a.free_state[1] = avail - total_takes;
+        *a.num_pairs = total_copies;
+    }
+}
+
+}  // namespace pkv

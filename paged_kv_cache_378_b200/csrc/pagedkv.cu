@@ -15,6 +15,7 @@
 #include "pkv_device.cuh"
 #include "kv_append.cuh"
 #include "block_copy.cuh"
+#include "block_manager.cuh"
 #include "attn_paged.cuh"
 
 namespace {
@@ -358,6 +359,39 @@ int attention_with_workspace(const pkv_cache_t* cache, int layer, const void* k_
     });
 }
 
+// Copy whole blocks from pool `src` to pool `dst` (the same cache for a
+// copy-on-write copy); d_num_pairs non-null: the count is read on the device
+// and num_pairs is its upper bound.
+int block_copy_launch(const pkv_cache_t* dst, const pkv_cache_t* src, const void* dst_k,
+                      const void* dst_v, const void* src_k, const void* src_v,
+                      const int32_t* src_dst_pairs, int num_pairs, const int32_t* d_num_pairs,
+                      void* stream) {
+    if (num_pairs < 0) return PKV_ERR_SHAPE;
+    if (num_pairs == 0) return PKV_OK;
+    if (!src_dst_pairs) return PKV_ERR_NULL;
+    const long long chunks = (long long)dst->num_kv_heads * dst->block_size * dst->head_dim / 8;
+    const long long total = (long long)num_pairs * dst->num_layers * 2 * chunks;
+    const long long want = (total + 256 * 4 - 1) / (256 * 4);   // four chunks per thread
+    const long long cap = (long long)device_sm_count() * 8;
+    const unsigned grid = (unsigned)(want < cap ? want : cap);
+    return launch_pdl(pkv::block_copy_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream,
+                      (uint4*)dst_k, (uint4*)dst_v, (const uint4*)src_k, (const uint4*)src_v,
+                      src_dst_pairs, num_pairs, dst->num_layers, src->num_blocks, dst->num_blocks,
+                      chunks, d_num_pairs);
+}
+
+// Device address of a host pool pointer: pinned (page-locked, mapped) host
+// memory only; null for pageable or device memory.
+const void* host_pool_device_ptr(const void* p) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (at.type != cudaMemoryTypeHost || !at.devicePointer) return nullptr;
+    return at.devicePointer;
+}
+
 }  // namespace
 
 extern "C" {
@@ -374,6 +408,7 @@ const char* pkv_strerror(int code) {
         case PKV_ERR_UNSUPPORTED: return "head_dim / block_size / group size not supported";
         case PKV_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
         case PKV_ERR_LAYER: return "layer index outside the cache";
+        case PKV_ERR_MEMORY: return "a host pool is not pinned, mapped host memory";
         case PKV_ERR_SCRATCH:
             return "request needs more scratch than the no-allocation buffer holds "
                    "(PKV_NOALLOC_SCRATCH_BYTES); use pkv_paged_decode_attention with a workspace";
@@ -407,19 +442,74 @@ int pkv_kv_append(const pkv_cache_t* cache, int layer, const void* k_new, const 
 
 int pkv_block_copy(const pkv_cache_t* cache, const int32_t* src_dst_pairs, int num_pairs,
                    void* stream) {
-    int rc = check_cache(cache);
+    const int rc = check_cache(cache);
     if (rc) return rc;
+    return block_copy_launch(cache, cache, cache->k_pool, cache->v_pool, cache->k_pool,
+                             cache->v_pool, src_dst_pairs, num_pairs, nullptr, stream);
+}
+
+int pkv_block_copy_device_count(const pkv_cache_t* cache, const int32_t* src_dst_pairs,
+                                int max_pairs, const int32_t* num_pairs, void* stream) {
+    const int rc = check_cache(cache);
+    if (rc) return rc;
+    if (!num_pairs && max_pairs > 0) return PKV_ERR_NULL;
+    return block_copy_launch(cache, cache, cache->k_pool, cache->v_pool, cache->k_pool,
+                             cache->v_pool, src_dst_pairs, max_pairs, num_pairs, stream);
+}
+
+int pkv_swap_blocks(const pkv_cache_t* device_cache, const pkv_cache_t* host_cache,
+                    const int32_t* src_dst_pairs, int num_pairs, int direction, void* stream) {
+    int rc = check_cache(device_cache);
+    if (rc) return rc;
+    rc = check_cache(host_cache);
+    if (rc) return rc;
+    if (direction != PKV_SWAP_OUT && direction != PKV_SWAP_IN) return PKV_ERR_SHAPE;
+    if (host_cache->num_layers != device_cache->num_layers ||
+        host_cache->num_kv_heads != device_cache->num_kv_heads ||
+        host_cache->block_size != device_cache->block_size ||
+        host_cache->head_dim != device_cache->head_dim)
+        return PKV_ERR_SHAPE;
     if (num_pairs < 0) return PKV_ERR_SHAPE;
     if (num_pairs == 0) return PKV_OK;
     if (!src_dst_pairs) return PKV_ERR_NULL;
-    const long long chunks = (long long)cache->num_kv_heads * cache->block_size * cache->head_dim / 8;
-    const long long total = (long long)num_pairs * cache->num_layers * 2 * chunks;
-    const long long want = (total + 256 * 4 - 1) / (256 * 4);   // four chunks per thread
-    const long long cap = (long long)device_sm_count() * 8;
-    const unsigned grid = (unsigned)(want < cap ? want : cap);
-    return launch_pdl(pkv::block_copy_kernel, dim3(grid), dim3(256), 0, (cudaStream_t)stream,
-                      reinterpret_cast<uint4*>(cache->k_pool), reinterpret_cast<uint4*>(cache->v_pool),
-                      src_dst_pairs, num_pairs, cache->num_layers, cache->num_blocks, chunks);
+    const void* hk = host_pool_device_ptr(host_cache->k_pool);
+    const void* hv = host_pool_device_ptr(host_cache->v_pool);
+    if (!hk || !hv) return PKV_ERR_MEMORY;
+    if (direction == PKV_SWAP_OUT)
+        return block_copy_launch(host_cache, device_cache, hk, hv, device_cache->k_pool,
+                                 device_cache->v_pool, src_dst_pairs, num_pairs, nullptr, stream);
+    return block_copy_launch(device_cache, host_cache, device_cache->k_pool, device_cache->v_pool,
+                             hk, hv, src_dst_pairs, num_pairs, nullptr, stream);
+}
+
+int pkv_block_manager_step(const pkv_block_state_t* st, int num_seqs, int max_blocks_per_seq,
+                           int num_blocks, int block_size, const int32_t* order,
+                           int64_t* slot_mapping, int32_t* copy_pairs, int32_t* num_pairs,
+                           void* stream) {
+    if (!st) return PKV_ERR_NULL;
+    if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || block_size <= 0)
+        return PKV_ERR_SHAPE;
+    if (num_seqs > pkv::BM_MAX_SEQS) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PKV_OK;
+    if (!st->block_tables || !st->seq_lens || !st->refcount || !st->free_ring || !st->free_state ||
+        !slot_mapping || !copy_pairs || !num_pairs)
+        return PKV_ERR_NULL;
+    pkv::BmArgs a;
+    a.block_tables = st->block_tables;
+    a.seq_lens = st->seq_lens;
+    a.refcount = st->refcount;
+    a.free_ring = st->free_ring;
+    a.free_state = st->free_state;
+    a.order = order;
+    a.slot_mapping = slot_mapping;
+    a.copy_pairs = copy_pairs;
+    a.num_pairs = num_pairs;
+    a.num_seqs = num_seqs;
+    a.max_blocks = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
+    a.block_size = block_size;
+    return launch_pdl(pkv::block_manager_kernel, dim3(1), dim3(pkv::BM_THREADS), 0,
+                      (cudaStream_t)stream, a);
 }
 
 int pkv_partition_tokens(int num_seqs, int num_kv_heads, int head_dim, int max_blocks_per_seq,

@@ -38,7 +38,7 @@ def test_library_loads_and_exports_every_declared_symbol():
 def test_version_and_error_strings():
     lib = pkv.library()
     assert lib.pkv_abi_version() == 1
-    for code in range(0, -8, -1):
+    for code in range(0, -10, -1):
         assert lib.pkv_strerror(code)
     assert b"unknown" in lib.pkv_strerror(-99)
 
@@ -92,6 +92,28 @@ def test_host_argument_checks_before_launch():
     assert fa(P(c), 0, 24, 16, 16, 2, 8, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -3
     assert fa(P(c), 0, 16, 16, 16, 2, 6, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -5
     assert fa(P(c), 0, 16, 16, 16, 0, 8, 16, 4, 16, 0.125, 16, None, 0, 0, None) == 0
+    # block copy with a device-side count: the count pointer is required
+    assert lib.pkv_block_copy_device_count(P(c), 16, 4, None, None) == -1
+    assert lib.pkv_block_copy_device_count(P(c), 16, 0, None, None) == 0
+    assert lib.pkv_block_copy_device_count(P(c), 16, -1, 16, None) == -2
+    # block swap: the host pool must match the device pool's shape; valid direction
+    sw = lib.pkv_swap_blocks
+    assert sw(P(c), P(_cache(head_dim=128)), 16, 1, 0, None) == -2
+    assert sw(P(c), P(_cache(num_layers=2)), 16, 1, 0, None) == -2
+    assert sw(P(c), P(_cache(num_blocks=3)), 16, 1, 2, None) == -2
+    assert sw(P(c), P(_cache(num_blocks=3)), 16, 0, 0, None) == 0
+    assert sw(P(c), P(_cache(num_blocks=3)), None, 2, 1, None) == -1
+    assert sw(P(c), P(_cache(k_pool=0)), 16, 1, 0, None) == -1
+    # device block manager step: state required, sizes checked, at most 4096 sequences
+    st = _lib.PkvBlockState(16, 16, 16, 16, 16)
+    bm = lib.pkv_block_manager_step
+    assert bm(None, 4, 8, 64, 16, None, 16, 16, 16, None) == -1
+    assert bm(P(st), -1, 8, 64, 16, None, 16, 16, 16, None) == -2
+    assert bm(P(st), 4, 0, 64, 16, None, 16, 16, 16, None) == -2
+    assert bm(P(st), 4097, 8, 64, 16, None, 16, 16, 16, None) == -5
+    assert bm(P(st), 0, 8, 64, 16, None, 16, 16, 16, None) == 0
+    assert bm(P(st), 4, 8, 64, 16, None, None, 16, 16, None) == -1
+    assert bm(P(_lib.PkvBlockState(16, 0, 16, 16, 16)), 4, 8, 64, 16, None, 16, 16, 16, None) == -1
 
 
 def test_workspace_and_partition_sizes():

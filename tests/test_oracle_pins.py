@@ -236,6 +236,33 @@ def test_block_copy_all_layers_only_pairs():
     assert np.array_equal(k3, kp) and np.array_equal(v3, vp)
 
 
+def test_swap_out_and_back_in_restores_every_byte():
+    # [AKIRA] 故事沒有說完的部分: blocks swapped out to host memory and brought back
+    # later.  Round trip through a host pool into other free device blocks gives
+    # the original bytes; the source pool is untouched; within one pool a swap is
+    # the (separately pinned) block copy.
+    rng = np.random.default_rng(12)
+    L, NB, NH, H, B, d = 2, 12, 6, 2, 4, 8
+    dk = _rand_bf16(rng, (L, NB, H, B, d))
+    dv = _rand_bf16(rng, (L, NB, H, B, d))
+    hk = np.zeros((L, NH, H, B, d), np.uint16)
+    hv = np.zeros((L, NH, H, B, d), np.uint16)
+    out = [(3, 0), (7, 5), (0, 2)]
+    hk2, hv2 = oa.swap_blocks(dk, dv, hk, hv, out)
+    for s, t in out:
+        assert np.array_equal(hk2[:, t], dk[:, s]) and np.array_equal(hv2[:, t], dv[:, s])
+    assert not hk2[:, [1, 3, 4]].any() and not hv2[:, [1, 3, 4]].any()
+    back = [(0, 9), (5, 10), (2, 11)]
+    dk2, dv2 = oa.swap_blocks(hk2, hv2, dk, dv, back)
+    for (s, _), (_, t) in zip(out, back):
+        assert np.array_equal(dk2[:, t], dk[:, s]) and np.array_equal(dv2[:, t], dv[:, s])
+    keep = [b for b in range(NB) if b not in (9, 10, 11)]
+    assert np.array_equal(dk2[:, keep], dk[:, keep]) and np.array_equal(dv2[:, keep], dv[:, keep])
+    same = oa.swap_blocks(dk, dv, dk, dv, [(1, 7), (4, 2)])
+    ref = oa.block_copy(dk, dv, [(1, 7), (4, 2)])
+    assert np.array_equal(same[0], ref[0]) and np.array_equal(same[1], ref[1])
+
+
 # ---------------------------------------------------------------------------
 # the merge rule
 # ---------------------------------------------------------------------------
