@@ -362,6 +362,42 @@ def block_manager_timing(pkv, w, device, iters=100):
     return sum(a.elapsed_time(b) for a, b in evs) / iters * 1e3
 
 
+def prefix_hash_timing(pkv, w, device, iters=50):
+    """Mean device time of hashing every full block of the batch (token ids
+    drawn per physical slot, so shared prompts share blocks); a memset queued
+    ahead of each launch hides the host's call overhead from the events."""
+    from workload import token_ids
+    tok = torch.from_numpy(token_ids(w)).to(device)
+    lens = torch.from_numpy(w.seq_lens).to(device)
+    N, T = tok.shape
+    mb = T // w.block_size
+    out = torch.zeros((N, mb), dtype=torch.int64, device=device)
+    busy = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    lib = pkv.library()
+    stream = torch.cuda.current_stream(device)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(iters)]
+    for i in range(iters + 3):
+        busy.zero_()
+        if i >= 3:
+            evs[i - 3][0].record(stream)
+        if lib.pkv_prefix_block_hashes(tok.data_ptr(), T, lens.data_ptr(), None, N, w.block_size,
+                                       out.data_ptr(), mb, sp):
+            raise SystemExit("prefix hash refused its arguments")
+        if i >= 3:
+            evs[i - 3][1].record(stream)
+    torch.cuda.synchronize(device)
+    if pkv.get_device_status(reset=True):
+        raise SystemExit("device status raised by the prefix hash")
+    us = sum(a.elapsed_time(b) for a, b in evs) / iters * 1e3
+    blocks = int(sum(int(n) // w.block_size for n in w.seq_lens))
+    return {"us": us, "full_blocks": blocks, "blocks_per_s": blocks / (us * 1e-6),
+            "token_bytes_gbs": blocks * w.block_size * 4 / (us * 1e-6) / 1e9,
+            "what": "FNV-1a 64 chain hash of every full block (parent hash, block tokens, "
+                    "extra key), one warp per sequence"}
+
+
 def swap_timing(pkv, w, device, blocks=1024, iters=10):
     """Block swap out to / back in from a pinned host pool: GB/s each way, and
     a plain pinned cudaMemcpy of the same bytes each way for reference."""
@@ -717,6 +753,7 @@ def main():
 
     bm_us = block_manager_timing(pkv, w, device) if w.num_seqs <= 4096 else None
     swap = swap_timing(pkv, w, device)
+    phash = prefix_hash_timing(pkv, w, device)
 
     peak, peak_kind = load_peak()
     q_out_bytes = 2 * w.num_seqs * spec.num_q_heads * spec.head_dim * 2
@@ -754,6 +791,7 @@ def main():
         "cpu_baseline": cpu,
         "e2e": e2e,
         "swap": swap,
+        "prefix_hash": phash,
         "block_manager": None if bm_us is None else {
             "us_per_step": bm_us, "num_seqs": w.num_seqs,
             "what": "device block-manager step (slot mapping, copy-on-write decisions, block "

@@ -170,6 +170,32 @@ int pkv_swap_blocks(const pkv_cache_t* device_cache, const pkv_cache_t* host_cac
                     const int32_t* src_dst_pairs, int num_pairs, int direction, void* stream);
 
 /*
+ * pkv_prefix_block_hashes -- hash every full block of every sequence, for
+ * finding cached prefix blocks again (automatic prefix caching).
+ *
+ * Defines ("Infra: PagedAttention", "共享前缀，分叉时 Copy-on-write", the
+ * paragraphs on Automatic Prefix Caching): only full blocks are cached; a
+ * block is reusable only when the whole prefix before it matches, so its
+ * hash covers the previous block's hash, the block's tokens and context
+ * identifiers such as a LoRA id.  The pages name no hash function; this one
+ * is FNV-1a 64 (h = 0xcbf29ce484222325, per byte h = (h ^ byte) *
+ * 0x100000001b3 mod 2^64):
+ *   digest c_b = FNV-1a(tokens of block b as int32 LE, extra key as uint64 LE)
+ *   hash   h_b = FNV-1a(h_{b-1} as uint64 LE, c_b as uint64 LE),  h_{-1} = 0
+ *
+ *   tokens       device int32 [num_seqs][max_tokens], token ids by position
+ *   seq_lens     device int32 [num_seqs]; blocks 0 .. seq_lens/B - 1 are hashed
+ *   extra_keys   device uint64 [num_seqs], or NULL for 0
+ *   hashes       device uint64 [num_seqs][max_blocks] out; entries past a
+ *                sequence's full blocks are not written
+ * A length above max_tokens, or more full blocks than max_blocks, sets
+ * PKV_DEV_LENGTH and is clamped.
+ */
+int pkv_prefix_block_hashes(const int32_t* tokens, int max_tokens, const int32_t* seq_lens,
+                            const uint64_t* extra_keys, int num_seqs, int block_size,
+                            uint64_t* hashes, int max_blocks, void* stream);
+
+/*
  * Block manager state on the device, for pkv_block_manager_step.  All device
  * pointers, owned by the caller.
  */

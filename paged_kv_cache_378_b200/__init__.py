@@ -29,7 +29,7 @@ from ._lib import PkvBlockState, PkvCache
 __all__ = [
     "PagedKVError", "kv_append", "block_copy", "paged_decode_attention",
     "append_paged_decode_attention", "BlockState", "block_manager_step", "swap_blocks",
-    "SWAP_OUT", "SWAP_IN",
+    "SWAP_OUT", "SWAP_IN", "prefix_block_hashes",
     "attention_workspace_bytes", "partition_tokens", "make_workspace",
     "get_device_status", "library", "DEV_RANGE", "DEV_LENGTH", "DEV_TIMEOUT", "DEV_NOBLOCKS",
 ]
@@ -135,6 +135,35 @@ def block_copy(src_dst_pairs, k_pool, v_pool, num_pairs=None, stream=None):
         rc = library().pkv_block_copy_device_count(ctypes.byref(cache), src_dst_pairs.data_ptr(),
                                                    n, num_pairs.data_ptr(), _stream(dev, stream))
     _check(rc, "block_copy")
+
+
+def prefix_block_hashes(tokens, seq_lens, block_size, extra_keys=None, max_blocks=None,
+                        stream=None):
+    """Hash of every full block of every sequence (FNV-1a 64 chain over the
+    parent hash, the block's tokens and the sequence's extra key).
+
+    ``tokens`` int32 CUDA ``[N, T]``; ``seq_lens`` int32 ``[N]``; ``extra_keys``
+    int64 ``[N]`` (bit patterns of uint64) or None.  Returns int64 ``[N,
+    max_blocks]`` holding the uint64 bit patterns; entries past a sequence's
+    full blocks are zero."""
+    dev = tokens.device
+    _need(tokens, "tokens", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    if tokens.dim() != 2 or seq_lens.shape != (tokens.shape[0],):
+        raise ValueError("tokens must be [N, T] and seq_lens [N]")
+    N, T = tokens.shape
+    if extra_keys is not None:
+        _need(extra_keys, "extra_keys", torch.int64, dev)
+        if extra_keys.shape != (N,):
+            raise ValueError("extra_keys must be [N]")
+    mb = T // int(block_size) if max_blocks is None else int(max_blocks)
+    out = torch.zeros((N, max(mb, 1)), dtype=torch.int64, device=dev)
+    rc = library().pkv_prefix_block_hashes(
+        tokens.data_ptr(), T, seq_lens.data_ptr(),
+        extra_keys.data_ptr() if extra_keys is not None else None, N, int(block_size),
+        out.data_ptr(), mb, _stream(dev, stream))
+    _check(rc, "prefix_block_hashes")
+    return out[:, :mb]
 
 
 SWAP_OUT = 0

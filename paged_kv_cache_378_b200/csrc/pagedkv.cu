@@ -16,6 +16,7 @@
 #include "kv_append.cuh"
 #include "block_copy.cuh"
 #include "block_manager.cuh"
+#include "prefix_hash.cuh"
 #include "attn_paged.cuh"
 
 namespace {
@@ -480,6 +481,21 @@ int pkv_swap_blocks(const pkv_cache_t* device_cache, const pkv_cache_t* host_cac
                                  device_cache->v_pool, src_dst_pairs, num_pairs, nullptr, stream);
     return block_copy_launch(device_cache, host_cache, device_cache->k_pool, device_cache->v_pool,
                              hk, hv, src_dst_pairs, num_pairs, nullptr, stream);
+}
+
+int pkv_prefix_block_hashes(const int32_t* tokens, int max_tokens, const int32_t* seq_lens,
+                            const uint64_t* extra_keys, int num_seqs, int block_size,
+                            uint64_t* hashes, int max_blocks, void* stream) {
+    if (num_seqs < 0 || max_tokens < 0 || max_blocks < 0 || block_size <= 0) return PKV_ERR_SHAPE;
+    if (num_seqs == 0 || max_blocks == 0) return PKV_OK;
+    if (!tokens || !seq_lens || !hashes) return PKV_ERR_NULL;
+    const int per_cta = 8;                                  // warps (sequences) per CTA
+    long long grid = ((long long)num_seqs + per_cta - 1) / per_cta;
+    const long long cap = (long long)device_sm_count() * 8;
+    if (grid > cap) grid = cap;
+    return launch_pdl(pkv::prefix_hash_kernel, dim3((unsigned)grid), dim3(per_cta * 32), 0,
+                      (cudaStream_t)stream, tokens, (long long)max_tokens, seq_lens, extra_keys,
+                      num_seqs, block_size, hashes, max_blocks);
 }
 
 int pkv_block_manager_step(const pkv_block_state_t* st, int num_seqs, int max_blocks_per_seq,

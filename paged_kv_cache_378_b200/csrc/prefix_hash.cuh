@@ -1,0 +1,82 @@
+// prefix_hash: hashes of every full KV block of every sequence, for finding
+// cached prefix blocks again.
+//
+// What it computes ("Infra: PagedAttention", section 共享前缀，分叉时
+// Copy-on-write, the paragraphs on Automatic Prefix Caching): only full
+// blocks are hashed, and a block's hash covers the hash of the block before
+// it, the block's tokens and a per-sequence context key (a LoRA id, say), so
+// equal hashes mean the whole prefix matches.  Definitions (the pages name no
+// function): FNV-1a 64 (Fowler, Noll, Vo): h = 0xcbf29ce484222325, per byte
+// h = (h ^ byte) * 0x100000001b3.  Block digest c_b = FNV-1a over the block's
+// tokens (int32, little-endian bytes) then the key (uint64, little-endian);
+// hash h_b = FNV-1a over h_{b-1} then c_b (uint64 LE each), h_{-1} = 0.
+//
+// One warp per sequence: the lanes hash the contents of 32 consecutive blocks
+// side by side, then every lane walks the short parent chain over those 32
+// digests (uniformly, from shuffles) and keeps its own block's hash.
+#pragma once
+
+#include "pkv_device.cuh"
+
+namespace pkv {
+
+constexpr uint64_t FNV64_OFFSET = 0xCBF29CE484222325ull;
+constexpr uint64_t FNV64_PRIME = 0x100000001B3ull;
+
+__device__ __forceinline__ uint64_t fnv_byte(uint64_t h, uint32_t b) { return (h ^ b) * FNV64_PRIME; }
+
+__device__ __forceinline__ uint64_t fnv_u32(uint64_t h, uint32_t v) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h = fnv_byte(h, (v >> (8 * i)) & 0xFFu);
+    return h;
+}
+
+__device__ __forceinline__ uint64_t fnv_u64(uint64_t h, uint64_t v) {
+    h = fnv_u32(h, (uint32_t)v);
+    return fnv_u32(h, (uint32_t)(v >> 32));
+}
+
+__global__ void __launch_bounds__(256)
+prefix_hash_kernel(const int32_t* __restrict__ tokens, long long row_stride,
+                   const int32_t* __restrict__ seq_lens, const uint64_t* __restrict__ extra_keys,
+                   int num_seqs, int block_size, uint64_t* __restrict__ hashes, int max_blocks) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int s = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); s < num_seqs; s += warps) {
+        long long len = __ldg(seq_lens + s);
+        if (len > row_stride) {
+            if (lane == 0) raise_status(PKV_DEV_LENGTH);
+            len = row_stride;
+        }
+        long long full = len > 0 ? len / block_size : 0;
+        if (full > max_blocks) {
+            if (lane == 0) raise_status(PKV_DEV_LENGTH);
+            full = max_blocks;
+        }
+        const uint64_t key = extra_keys ? __ldg(extra_keys + s) : 0ull;
+        const int32_t* row = tokens + (size_t)s * row_stride;
+        uint64_t parent = 0;
+        for (long long b0 = 0; b0 < full; b0 += 32) {
+            const long long b = b0 + lane;
+            uint64_t c = 0;
+            if (b < full) {
+                uint64_t h = FNV64_OFFSET;
+                const int32_t* t = row + b * block_size;
+                for (int i = 0; i < block_size; ++i) h = fnv_u32(h, (uint32_t)__ldg(t + i));
+                c = fnv_u64(h, key);
+            }
+            const int n = full - b0 < 32 ? (int)(full - b0) : 32;
+            uint64_t mine = 0;
+            for (int j = 0; j < n; ++j) {
+                const uint64_t cj = __shfl_sync(0xFFFFFFFFu, c, j);
+                parent = fnv_u64(fnv_u64(FNV64_OFFSET, parent), cj);
+                if (lane == j) mine = parent;
+            }
+            if (b < full) hashes[(size_t)s * max_blocks + b] = mine;
+        }
+    }
+}
+
+}  // namespace pkv

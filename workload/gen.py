@@ -227,3 +227,28 @@ def make_workload(key_or_spec, block_size=None, seed=None, device="cpu", values=
             if poison:
                 pool[layer].masked_fill_(dead, nan_bits)
     return w
+
+
+def token_ids(w, vocab=128256, seed=None):
+    """Token id of every position of every sequence, int32 ``[N, max_blocks*B]``
+    (zero past each length), for the prefix-hash workload.
+
+    Ids are drawn per physical slot (uniform over a Llama-3-sized vocabulary)
+    and read through each sequence's table, so sequences that share a physical
+    block share its tokens, as a shared prompt does.  A copy-on-write
+    destination holds its source's tokens; each appended token gets its own id.
+    Input generation only.
+    """
+    rng = np.random.default_rng(w.seed + 1000 if seed is None else seed)
+    B = w.block_size
+    slot_tok = rng.integers(0, vocab, w.num_blocks * B).astype(np.int32)
+    for src, dst in w.copy_pairs.tolist():
+        slot_tok[dst * B:(dst + 1) * B] = slot_tok[src * B:(src + 1) * B]
+    slot_tok[w.slot_mapping] = rng.integers(0, vocab, w.num_seqs).astype(np.int32)
+    N, maxb = w.block_tables.shape
+    out = np.zeros((N, maxb * B), np.int32)
+    for s in range(N):
+        n = int(w.seq_lens[s])
+        pos = np.arange(n)
+        out[s, :n] = slot_tok[w.block_tables[s, pos // B].astype(np.int64) * B + pos % B]
+    return out
