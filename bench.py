@@ -779,7 +779,8 @@ def main():
                             if gs.fused else
                             "block_copy, then per layer kv_append and attention launches")},
         "pct_hbm_peak": 100.0 * value / peak,
-        "decode_tokens_per_s_per_layer": seqs_total / (ms_per_step * 1e-3),
+        # one token per sequence per layer: N x L tokens cross a layer per step
+        "decode_tokens_per_s_per_layer": seqs_total * spec.num_layers / (ms_per_step * 1e-3),
         "kv_bytes_per_step": {"unique": unique_bytes * spec.num_layers,
                               "logical": logical_bytes * spec.num_layers},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
