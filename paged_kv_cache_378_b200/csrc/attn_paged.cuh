@@ -64,6 +64,7 @@ struct AttnArgs {
     float2* part_mz;               // [R_max][2][G]    (m, Z) of a partial, base 2
     float* part_o;                 // [R_max][2][G][D] unnormalised partial output
     unsigned int* tickets;         // [N*Hkv] zero at rest
+    unsigned int* group_tickets;   // [R_max][2] zero at rest: a group's first range and slot
     long long* prefix_g;           // [N+1] tile prefix, used when N > PREFIX_SMEM
     int R_max;                     // ranges the workspace holds
     // fused append (k_new != nullptr): the new token of sequence s, at
@@ -482,102 +483,140 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const long long au = m.f - m.t;                    // the unit's first flat tile
         const long long r_lo = sc.range_of(au);
         const long long r_hi = sc.range_of(au + nt - 1);
-        const unsigned others = (unsigned)(r_hi - r_lo);   // pieces in other ranges
         // partial slot of range j: 0 if the unit began in an earlier range
         auto piece_row = [&](long long j) -> size_t {
             return ((size_t)j * 2 + ((au < sc.begin(j)) ? 0 : 1)) * G + g_row;
         };
-        auto store_mine = [&]() {
+        // Two levels when a unit has many pieces: groups of GR consecutive
+        // ranges merge first (their result goes to the slot of the group's
+        // first range), then the groups merge.  A warp folds at most GR + the
+        // number of groups pieces one after another instead of every piece.
+        constexpr int GR = 8;
+        const long long P = r_hi - r_lo + 1;
+        const long long NG = (P + GR - 1) / GR;
+        const long long kg = (m.r - r_lo) / GR;             // this piece's group
+        float M = ws.m, Z = l;                              // this piece's state (row of the lane)
+        auto store_state = [&](size_t pr) {
             if (g_row < G) {
-                const size_t pr = piece_row(m.r);
                 float* po = a.part_o + pr * D + 2 * c4;
 #pragma unroll
                 for (int n = 0; n < D / 8; ++n)
                     st_cg(reinterpret_cast<float2*>(po + 8 * n), make_float2(ws.o[n][0], ws.o[n][1]));
-                if (c4 == 0) st_cg(a.part_mz + pr, make_float2(ws.m, l));
+                if (c4 == 0) st_cg(a.part_mz + pr, make_float2(M, Z));
             }
         };
-        // Every other piece already counted on the ticket: this piece is the
-        // last and merges without publishing itself.  Otherwise publish, count,
-        // and merge only if the count makes this piece the last.
-        unsigned seen = 0;
-        if (lane == 0) seen = ld_acquire(a.tickets + unit);
-        seen = __shfl_sync(FULL, seen, 0);
-        bool mine_in_memory = false;
-        if (seen != others) {
-            store_mine();
-            __threadfence();
-            __syncwarp();
-            unsigned prev = 0;
-            if (lane == 0) prev = atomicAdd(a.tickets + unit, 1u);
-            prev = __shfl_sync(FULL, prev, 0);
-            if (prev != others) return;                   // not the last piece
-            __threadfence();
-            mine_in_memory = true;
-        }
-        if (lane == 0) st_cg(reinterpret_cast<int*>(a.tickets) + unit, 0);   // ready for the next launch
-        // Fold the pieces in range order into this lane's row of the register
-        // state: (M, Z, o) <- (M', e^{M-M'} Z + e^{m_j-M'} Z_j, e^{M-M'} o + e^{m_j-M'} o_j),
-        // M' = max(M, m_j).  The order is fixed, so the result does not depend
-        // on which piece merges.  When this piece is not the first, it goes to
-        // memory and the fold starts from the first piece.
-        float M = ws.m, Z = l;
-        long long j0 = r_lo + 1;
-        if (m.r != r_lo) {
-            if (!mine_in_memory) store_mine();
-            __syncwarp();
-            if (g_row < G) {
-                const size_t pr = piece_row(r_lo);
-                const float* po = a.part_o + pr * D + 2 * c4;
-#pragma unroll
-                for (int n = 0; n < D / 8; ++n) {
-                    const float2 v = ld_cg(reinterpret_cast<const float2*>(po + 8 * n));
-                    ws.o[n][0] = v.x;
-                    ws.o[n][1] = v.y;
-                }
-                const float2 mz = ld_cg(a.part_mz + pr);
-                M = mz.x;
-                Z = mz.y;
-            }
-        }
-        // head_dim 64: the next piece's loads are issued before this one is
+        // head_dim 64: the next element's loads are issued before this one is
         // folded in; head_dim 128 has no registers to spare for that
         constexpr bool PREFETCH = D == 64;
-        float2 v[D / 8], mz = make_float2(0.f, 0.f);
-        auto fetch = [&](long long j) {
-            if (g_row < G) {
-                const size_t pr = piece_row(j);
-                const float* po = a.part_o + pr * D + 2 * c4;
-#pragma unroll
-                for (int n = 0; n < D / 8; ++n) v[n] = ld_cg(reinterpret_cast<const float2*>(po + 8 * n));
-                mz = ld_cg(a.part_mz + pr);
-            }
+        // One merge level over elements first..last (slot_of(e): the element's
+        // partial row), this warp holding element `mine` in registers.  Every
+        // other element already counted on the ticket: this warp is the last
+        // and merges without publishing its own.  Otherwise publish, count,
+        // and merge only if the count makes it the last.  The fold runs in
+        // element order from the first element, so the result does not depend
+        // on which warp merges:
+        //   (M, Z, o) <- (M', e^{M-M'} Z + e^{m_e-M'} Z_e, e^{M-M'} o + e^{m_e-M'} o_e),
+        //   M' = max(M, m_e).
+        // Returns false when another warp will merge.
+        // element e's partial row: range e, or (groups) the first range of group e
+        auto slot_of_level = [&](long long e, bool groups) -> size_t {
+            return piece_row(groups ? r_lo + e * GR : e);
         };
-        if (PREFETCH && j0 <= r_hi) fetch(j0);
-        for (long long j = j0; j <= r_hi; ++j) {
-            float2 w[D / 8], wz;
-            if (PREFETCH) {
-#pragma unroll
-                for (int n = 0; n < D / 8; ++n) w[n] = v[n];
-                wz = mz;
-                if (j < r_hi) fetch(j + 1);
-            } else {
-                fetch(j);
-#pragma unroll
-                for (int n = 0; n < D / 8; ++n) w[n] = v[n];
-                wz = mz;
+        auto merge_level = [&](long long first, long long last, long long mine, unsigned* ticket,
+                               bool groups) -> bool {
+            auto slot_of = [&](long long e) -> size_t { return slot_of_level(e, groups); };
+            const unsigned others = (unsigned)(last - first);
+            unsigned seen = 0;
+            if (lane == 0) seen = ld_acquire(ticket);
+            seen = __shfl_sync(FULL, seen, 0);
+            bool stored = false;
+            if (seen != others) {
+                store_state(slot_of(mine));
+                __threadfence();
+                __syncwarp();
+                unsigned prev = 0;
+                if (lane == 0) prev = atomicAdd(ticket, 1u);
+                prev = __shfl_sync(FULL, prev, 0);
+                if (prev != others) return false;           // not the last
+                __threadfence();
+                stored = true;
             }
-            if (g_row < G) {
-                const float mx = fmaxf(M, wz.x);
-                const float ca = fast_exp2(M - mx), cb = fast_exp2(wz.x - mx);
-                Z = fmaf(cb, wz.y, Z * ca);
-                M = mx;
+            if (lane == 0) st_cg(reinterpret_cast<int*>(ticket), 0);   // ready for the next launch
+            if (mine != first) {                            // the fold starts from the first element
+                if (!stored) store_state(slot_of(mine));
+                __syncwarp();
+                if (g_row < G) {
+                    const size_t pr = slot_of(first);
+                    const float* po = a.part_o + pr * D + 2 * c4;
 #pragma unroll
-                for (int n = 0; n < D / 8; ++n) {
-                    ws.o[n][0] = fmaf(cb, w[n].x, ws.o[n][0] * ca);
-                    ws.o[n][1] = fmaf(cb, w[n].y, ws.o[n][1] * ca);
+                    for (int n = 0; n < D / 8; ++n) {
+                        const float2 v = ld_cg(reinterpret_cast<const float2*>(po + 8 * n));
+                        ws.o[n][0] = v.x;
+                        ws.o[n][1] = v.y;
+                    }
+                    const float2 mz = ld_cg(a.part_mz + pr);
+                    M = mz.x;
+                    Z = mz.y;
                 }
             }
+            float2 v[D / 8], mz = make_float2(0.f, 0.f);
+            auto fetch = [&](long long e) {
+                if (g_row < G) {
+                    const size_t pr = slot_of(e);
+                    const float* po = a.part_o + pr * D + 2 * c4;
+#pragma unroll
+                    for (int n = 0; n < D / 8; ++n) v[n] = ld_cg(reinterpret_cast<const float2*>(po + 8 * n));
+                    mz = ld_cg(a.part_mz + pr);
+                }
+            };
+            if (PREFETCH && first < last) fetch(first + 1);
+            for (long long e = first + 1; e <= last; ++e) {
+                float2 w[D / 8], wz;
+                if (PREFETCH) {
+#pragma unroll
+                    for (int n = 0; n < D / 8; ++n) w[n] = v[n];
+                    wz = mz;
+                    if (e < last) fetch(e + 1);
+                } else {
+                    fetch(e);
+#pragma unroll
+                    for (int n = 0; n < D / 8; ++n) w[n] = v[n];
+                    wz = mz;
+                }
+                if (g_row < G) {
+                    const float mx = fmaxf(M, wz.x);
+                    const float ca = fast_exp2(M - mx), cb = fast_exp2(wz.x - mx);
+                    Z = fmaf(cb, wz.y, Z * ca);
+                    M = mx;
+#pragma unroll
+                    for (int n = 0; n < D / 8; ++n) {
+                        ws.o[n][0] = fmaf(cb, w[n].x, ws.o[n][0] * ca);
+                        ws.o[n][1] = fmaf(cb, w[n].y, ws.o[n][1] * ca);
+                    }
+                }
+            }
+            return true;
+        };
+        // level 1: the pieces of this piece's group (all pieces when there is
+        // one group); level 2: the groups, whose results sit in the slots of
+        // their first ranges.  One call site, so the merge is inlined once.
+        long long first = r_lo + kg * GR;
+        long long last = first + GR - 1 < r_hi ? first + GR - 1 : r_hi;
+        long long mine = m.r;
+        // a group is named by its first range and this unit's slot in it (a
+        // range starts groups of at most two units: the one it continues and
+        // the one it starts)
+        unsigned* ticket = NG == 1 ? a.tickets + unit
+                                   : a.group_tickets + first * 2 + ((au < sc.begin(first)) ? 0 : 1);
+        bool groups = false;
+        for (int level = 0;; ++level) {
+            if (!merge_level(first, last, mine, ticket, groups)) return;
+            if (NG == 1 || level == 1) break;
+            first = 0;
+            last = NG - 1;
+            mine = kg;
+            ticket = a.tickets + unit;
+            groups = true;
         }
         if (g_row < G) {
             const float inv = 1.0f / Z;

@@ -114,7 +114,7 @@ constexpr int attn_stages() {
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WorkspaceLayout {
-    size_t prefix_off, mz_off, o_off, tickets_off, total;
+    size_t prefix_off, mz_off, o_off, tickets_off, gtickets_off, total;
     int R_max;
     int cap_tiles;
 };
@@ -131,7 +131,8 @@ bool fill_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, 
     w->mz_off = N > (size_t)pkv::PREFIX_SMEM ? align_up((N + 1) * sizeof(long long), 256) : 0;
     w->o_off = w->mz_off + align_up((size_t)r_max * 2 * G * sizeof(float2), 256);
     w->tickets_off = w->o_off + align_up((size_t)r_max * 2 * G * head_dim * sizeof(float), 256);
-    w->total = w->tickets_off + align_up(N * num_kv_heads * sizeof(unsigned int), 256);
+    w->gtickets_off = w->tickets_off + align_up(N * num_kv_heads * sizeof(unsigned int), 256);
+    w->total = w->gtickets_off + align_up((size_t)r_max * 2 * sizeof(unsigned int), 256);
     return true;
 }
 
@@ -346,6 +347,7 @@ int attention_with_workspace(const pkv_cache_t* cache, int layer, const void* k_
     a.part_mz = reinterpret_cast<float2*>(ws + w.mz_off);
     a.part_o = reinterpret_cast<float*>(ws + w.o_off);
     a.tickets = reinterpret_cast<unsigned int*>(ws + w.tickets_off);
+    a.group_tickets = reinterpret_cast<unsigned int*>(ws + w.gtickets_off);
     a.prefix_g = reinterpret_cast<long long*>(ws + w.prefix_off);
     a.R_max = w.R_max;
     a.k_new = static_cast<const uint4*>(k_new);
@@ -622,6 +624,7 @@ int pkv_paged_decode_attention_noalloc(const pkv_cache_t* cache, int layer, cons
     a.part_mz = reinterpret_cast<float2*>(ws + w.mz_off);
     a.part_o = reinterpret_cast<float*>(ws + w.o_off);
     a.tickets = reinterpret_cast<unsigned int*>(ws + w.tickets_off);
+    a.group_tickets = reinterpret_cast<unsigned int*>(ws + w.gtickets_off);
     a.prefix_g = reinterpret_cast<long long*>(ws + w.prefix_off);
     a.k_new = nullptr;                                // no fused append here
     a.v_new = nullptr;
