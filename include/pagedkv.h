@@ -241,11 +241,11 @@ int pkv_block_manager_step(const pkv_block_state_t* state, int num_seqs,
 
 /*
  * pkv_attention_workspace_bytes -- bytes of workspace pkv_paged_decode_attention
- * needs for these sizes on the current device: the work plan (a prefix of
- * tiles per sequence and the start of every work range), the partial results
- * of sequences split across ranges, and one ticket per (sequence, kv head).
- * `partition_tokens` as passed to the attention call.  Returns 0 for invalid
- * sizes.
+ * needs for these sizes on the current device: the tile prefix per sequence
+ * (batches over 768 sequences; smaller ones keep it in shared memory), the
+ * partial results of sequences split across ranges, one ticket per (sequence,
+ * kv head) and one per group of ranges.  `partition_tokens` as passed to the
+ * attention call.  Returns 0 for invalid sizes.
  */
 size_t pkv_attention_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,
                                      int head_dim, int max_blocks_per_seq, int block_size,
@@ -356,8 +356,8 @@ int pkv_append_paged_decode_attention(const pkv_cache_t* cache, int layer,
  * moment).
  *
  * Same arguments and result as pkv_paged_decode_attention, without a
- * workspace: the scratch (partial results of split sequences, one ticket per
- * (sequence, kv head), the tile prefix of batches over 1024 sequences) lives
+ * workspace: the scratch (partial results of split sequences, their tickets,
+ * the tile prefix of batches over 768 sequences) lives
  * in one fixed device array of PKV_NOALLOC_SCRATCH_BYTES (16 MiB) inside this
  * library.  Every GPU that loads the library holds that array until the
  * process exits.  The call itself allocates nothing: no cudaMalloc, no
