@@ -70,7 +70,7 @@ def load_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def load_traffic(workload_key, block_size, fused):
+def load_traffic(workload_key, block_size, step):
     """DRAM bytes per attention launch from the committed ncu summary, or None
     if absent, for another workload or step, or taken on different kernel source."""
     try:
@@ -80,7 +80,7 @@ def load_traffic(workload_key, block_size, fused):
         return None
     for r in rec.get("captures", []):
         if r.get("workload") == workload_key and int(r.get("block_size", -1)) == block_size \
-                and bool(r.get("fused", False)) == fused \
+                and r.get("step") == step \
                 and r.get("kernel_source_hash") == kernel_source_hash():
             return r.get("dram_bytes_per_launch")
     return None
@@ -208,7 +208,7 @@ class GpuStep:
     device time of a step.
     """
 
-    def __init__(self, pkv, w, replicas, partition, device, fused=True):
+    def __init__(self, pkv, w, replicas, partition, device, mode="cow"):
         from paged_kv_cache_378_b200._lib import PkvCache
         self.lib = pkv.library()
         spec = w.spec
@@ -232,16 +232,25 @@ class GpuStep:
         self.slots = torch.from_numpy(w.slot_mapping).to(device)
         self.pairs = torch.from_numpy(w.copy_pairs).to(device)
         self.npairs = int(w.copy_pairs.shape[0])
+        self.cow = torch.from_numpy(cow_sources(w)).to(device)
         self.out = torch.empty_like(w.q)
         self.resident = dict(q=self.q, k_new=self.k_new, v_new=self.v_new, tables=self.tables,
-                             lens=self.lens, slots=self.slots, pairs=self.pairs, out=self.out)
+                             lens=self.lens, slots=self.slots, pairs=self.pairs, cow=self.cow,
+                             out=self.out)
+        if mode not in ("cow", "fused", "two-call"):
+            raise ValueError(f"unknown step mode {mode}")
+        self.mode = mode
+        # what a step reads from its inputs (the end-to-end run uploads these)
+        self.input_keys = ["q", "k_new", "v_new", "tables", "lens"] + (
+            ["cow"] if mode == "cow" else ["pairs"] + (["slots"] if mode == "two-call" else []))
         self.partition = int(partition)
         self.ws = pkv.make_workspace(self.N, self.Hq, H, D, w.max_blocks, B, self.partition,
                                      device=device)
         self.scale = ctypes.c_float(spec.scale)
         self.maxb = w.max_blocks
-        self.fused = fused
-        self.launches_per_step = (1 if self.npairs else 0) + (1 if fused else 2) * self.L
+        self.fused = mode != "two-call"
+        self.launches_per_step = ((1 if self.npairs and mode != "cow" else 0)
+                                  + (2 if mode == "two-call" else 1) * self.L)
 
     def run(self, step_index, evl=None, bufs=None):
         """Launch one step; ``evl`` = per-layer (start, end) events around
@@ -251,14 +260,15 @@ class GpuStep:
         b = bufs if bufs is not None else self.resident
         _, cref = self.caches[step_index % len(self.caches)]
         rc = 0
-        if self.npairs:
+        if self.npairs and self.mode != "cow":
             rc |= lib.pkv_block_copy(cref, b["pairs"].data_ptr(), self.npairs, self.sp)
+        cow = b["cow"].data_ptr() if self.mode == "cow" else None
         for layer in range(self.L):
-            if self.fused:                   # append of the new token fused into attention
+            if self.fused:                   # append (and copy-on-write) fused into attention
                 if evl is not None:
                     evl[layer][0].record(self.stream)
                 rc |= lib.pkv_append_paged_decode_attention(
-                    cref, layer, b["k_new"][layer].data_ptr(), b["v_new"][layer].data_ptr(),
+                    cref, layer, b["k_new"][layer].data_ptr(), b["v_new"][layer].data_ptr(), cow,
                     b["q"][layer].data_ptr(), self.N, self.Hq, b["tables"].data_ptr(), self.maxb,
                     b["lens"].data_ptr(), self.scale, b["out"][layer].data_ptr(),
                     self.ws.data_ptr(), self.ws.numel(), self.partition, self.sp)
@@ -289,6 +299,14 @@ def packed_buffers(like, device, pin):
     views = {k: raw[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
              for (k, t), o in zip(like.items(), offs.values())}
     return raw, views
+
+
+def cow_sources(w):
+    """Per sequence, the source block of this step's copy-on-write (-1 if
+    none): the pair whose destination is the sequence's tail block."""
+    src_of = {int(d): int(s) for s, d in w.copy_pairs}
+    tails = w.block_tables[np.arange(w.num_seqs), (w.seq_lens.astype(np.int64) - 1) // w.block_size]
+    return np.array([src_of.get(int(t), -1) for t in tails], np.int32)
 
 
 def prestep_state(w):
@@ -343,7 +361,7 @@ def block_manager_timing(pkv, w, device, iters=100):
     sp = ctypes.c_void_p(stream.cuda_stream)
     args = (ctypes.byref(c), N, maxb, int(w.num_blocks), int(w.block_size),
             order.data_ptr() if order is not None else None, slots.data_ptr(), pairs.data_ptr(),
-            npairs.data_ptr(), sp)
+            npairs.data_ptr(), None, sp)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(iters)]
     for i in range(iters + 5):
@@ -441,8 +459,9 @@ def swap_timing(pkv, w, device, blocks=1024, iters=10):
 
 def e2e_run(pkv, w, gs, steps, device):
     """The same step through the C ABI from host buffers.  Every step uploads
-    its inputs (q, k_new, v_new, block tables, lengths, slot mapping, copy
-    pairs: one packed pinned buffer, one copy) and reads its attention output
+    its inputs (what the step reads: q, k_new, v_new, block tables, lengths,
+    and the copy sources, or the copy pairs and slot mapping; one packed
+    pinned buffer, one copy) and reads its attention output
     back to pinned host memory.  Two buffer sets alternate, so step i+1's
     upload and step i-1's download run on copy streams while step i computes."""
     # host threads and pinned buffers on the GPU's NUMA node: copies then
@@ -450,9 +469,11 @@ def e2e_run(pkv, w, gs, steps, device):
     local = gpu_local_cpus(pci_bus_id(device.index if device.index is not None else 0))
     if local:
         os.sched_setaffinity(0, local)
-    host_src = dict(q=w.q.cpu(), k_new=w.k_new.cpu(), v_new=w.v_new.cpu(),
-                    tables=torch.from_numpy(w.block_tables), lens=torch.from_numpy(w.seq_lens),
-                    slots=torch.from_numpy(w.slot_mapping), pairs=torch.from_numpy(w.copy_pairs))
+    every = dict(q=w.q.cpu(), k_new=w.k_new.cpu(), v_new=w.v_new.cpu(),
+                 tables=torch.from_numpy(w.block_tables), lens=torch.from_numpy(w.seq_lens),
+                 slots=torch.from_numpy(w.slot_mapping), pairs=torch.from_numpy(w.copy_pairs),
+                 cow=torch.from_numpy(cow_sources(w)))
+    host_src = {k: every[k] for k in gs.input_keys}
     h_raw, h_views = packed_buffers(host_src, "cpu", True)
     for k, t in host_src.items():
         h_views[k].copy_(t)
@@ -639,8 +660,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--soak-seconds", type=float, default=1.5)
-    ap.add_argument("--two-call", action="store_true",
-                    help="kv_append and attention as two launches per layer (default: one fused launch)")
+    ap.add_argument("--step", choices=["cow", "fused", "two-call"], default="cow",
+                    help="cow (default): one launch per layer doing copy-on-write, append and "
+                         "attention; fused: block_copy, then append+attention per layer; "
+                         "two-call: block_copy, then kv_append and attention per layer")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -683,7 +706,7 @@ def main():
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     nrep = max(1, min(16, math.ceil(4 * l2 / pool_bytes)))
     replicas = [(w.k_pool, w.v_pool)] + [(w.k_pool.clone(), w.v_pool.clone()) for _ in range(nrep - 1)]
-    gs = GpuStep(pkv, w, replicas, part, device, fused=not args.two_call)
+    gs = GpuStep(pkv, w, replicas, part, device, mode=args.step)
     pkv.get_device_status(reset=True)
 
     # warm-up
@@ -693,10 +716,14 @@ def main():
     if pkv.get_device_status(reset=True):
         raise SystemExit("device status raised during warm-up")
 
-    # Attention is bracketed by events on every EVENT_EVERY-th step only: an
+    # When the attention kernel is the only kernel of the step (copy-on-write
+    # folded in), every launch in the timed region is that kernel and its
+    # average duration is the timed region over the launches.  Otherwise
+    # attention is bracketed by events on every EVENT_EVERY-th step only: an
     # event between two kernels ends their programmatic overlap, so the other
     # steps run chained as a user's stream would.
-    ev_steps = list(range(0, args.steps, EVENT_EVERY))
+    only_attention = gs.mode == "cow"
+    ev_steps = [] if only_attention else list(range(0, args.steps, EVENT_EVERY))
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(len(ev_steps) * spec.num_layers)]
     t_start = torch.cuda.Event(enable_timing=True)
@@ -732,7 +759,12 @@ def main():
     if status:
         raise SystemExit(f"device status {status:#x} raised in the timed region")
 
-    attn_ms = [a.elapsed_time(b) for a, b in evs]
+    if only_attention:
+        attn_ms = [ms / (args.steps * spec.num_layers)] * (args.steps * spec.num_layers)
+        sampling = "every launch in the timed region is this kernel: timed region / launches"
+    else:
+        attn_ms = [a.elapsed_time(b) for a, b in evs]
+        sampling = f"attention bracketed on every {EVENT_EVERY}th timed step"
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
 
     # totals over ranks: device time is the max, work is the sum
@@ -760,9 +792,13 @@ def main():
     meta_bytes = w.block_tables.nbytes + w.seq_lens.nbytes
     # the fused kernel also reads k_new/v_new and stores them in their slots
     append_bytes = 2 * (2 * w.num_seqs * spec.num_kv_heads * spec.head_dim * 2) if gs.fused else 0
-    alg_bytes = unique_bytes + q_out_bytes + meta_bytes + append_bytes
+    # with the copy-on-write folded in, the kernel also writes each copied tail
+    # block (this layer, K and V); its source is read as the tail itself
+    cow_bytes = (gs.npairs * spec.num_kv_heads * B * spec.head_dim * 2 * 2
+                 if gs.mode == "cow" else 0)
+    alg_bytes = unique_bytes + q_out_bytes + meta_bytes + append_bytes + cow_bytes
     achieved = alg_bytes / (attn_avg_ms * 1e-3) / 1e9
-    traffic = load_traffic(args.workload, B, gs.fused)
+    traffic = load_traffic(args.workload, B, gs.mode)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -775,9 +811,11 @@ def main():
                    "l2": f"inputs larger than L2: {nrep} rotating copies of the KV pools, "
                          f"{nrep * pool_bytes / 1e9:.2f} GB vs {l2 / 1e6:.0f} MB L2",
                    "parallelism": f"dp{world} (independent batches, no collective)",
-                   "step": ("block_copy, then per layer one fused append+attention launch"
-                            if gs.fused else
-                            "block_copy, then per layer kv_append and attention launches")},
+                   "step": {"cow": "per layer one launch: copy-on-write of shared tails, "
+                                   "append of the new token, attention",
+                            "fused": "block_copy, then per layer one fused append+attention launch",
+                            "two-call": "block_copy, then per layer kv_append and attention "
+                                        "launches"}[gs.mode]},
         "pct_hbm_peak": 100.0 * value / peak,
         # one token per sequence per layer: N x L tokens cross a layer per step
         "decode_tokens_per_s_per_layer": seqs_total * spec.num_layers / (ms_per_step * 1e-3),
@@ -788,7 +826,7 @@ def main():
                      "kernel": "paged_attention_kernel", "alg_bytes_per_launch": alg_bytes,
                      "avg_launch_us": attn_avg_ms * 1e3, "peak_source": f"{peak_kind} hbm_gbs",
                      "timed_launches": len(attn_ms),
-                     "event_sampling": f"attention bracketed on every {EVENT_EVERY}th timed step"},
+                     "event_sampling": sampling},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "swap": swap,

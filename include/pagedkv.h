@@ -26,11 +26,13 @@
  *    may start while the kernel before it on the stream finishes, and waits
  *    for that kernel to complete before it reads or writes the pools, q,
  *    k_new, v_new, the tables, the workspace or out.  The one exception:
- *    the attention kernel reads seq_lens before that wait, so seq_lens
- *    must be written by copies or kernels that do not release their
- *    dependents early (cudaTriggerProgrammaticLaunchCompletion): such a
- *    writer could still be running when the attention kernel starts.  No
- *    kernel of this library writes seq_lens.
+ *    the attention kernels read seq_lens and block_tables before that wait
+ *    (to plan their work), so those two must be written by copies or by
+ *    kernels that do not release their dependents early
+ *    (cudaTriggerProgrammaticLaunchCompletion): such a writer could still
+ *    be running when the attention kernel starts.  The one kernel of this
+ *    library that writes them, pkv_block_manager_step, does not release
+ *    early.
  *  - Return value: PKV_OK, or a negative PKV_ERR_* code when an argument
  *    check fails on the host (nothing is launched) or a launch fails.
  *  - Faults found by the kernels themselves (a block id or slot outside the
@@ -227,6 +229,9 @@ typedef struct pkv_block_state {
  *                  token (block * block_size + offset)
  *   copy_pairs     device int32 [num_seqs][2] out, (src, dst) in writer order
  *   num_pairs      device int32 [1] out
+ *   cow_src        device int32 [num_seqs] out, or NULL: per sequence the
+ *                  source block of its copy (-1 if it does not copy), the
+ *                  form pkv_append_paged_decode_attention takes
  * On return the tables, lengths (+1), counts and free state are updated.
  * num_seqs <= 4096 (PKV_ERR_UNSUPPORTED above).  If the free blocks do not
  * suffice, or an order entry, a length or a tail block id is out of range,
@@ -237,7 +242,8 @@ typedef struct pkv_block_state {
 int pkv_block_manager_step(const pkv_block_state_t* state, int num_seqs,
                            int max_blocks_per_seq, int num_blocks, int block_size,
                            const int32_t* order, int64_t* slot_mapping,
-                           int32_t* copy_pairs, int32_t* num_pairs, void* stream);
+                           int32_t* copy_pairs, int32_t* num_pairs, int32_t* cow_src,
+                           void* stream);
 
 /*
  * pkv_attention_workspace_bytes -- bytes of workspace pkv_paged_decode_attention
@@ -328,6 +334,17 @@ int pkv_paged_decode_attention(const pkv_cache_t* cache, int layer,
  *                  the table gives for position seq_lens[s] - 1, i.e. block
  *                  block_tables[s][(seq_lens[s]-1)/B], row (seq_lens[s]-1)%B;
  *                  sequences with seq_lens[s] == 0 append nothing.
+ *   cow_src        device int32 [num_seqs], or NULL: the copy-on-write of
+ *                  the step folded into this launch.  cow_src[s] >= 0 means
+ *                  the sequence's tail block (the table's block for position
+ *                  seq_lens[s] - 1) is a fresh copy of block cow_src[s]: this
+ *                  launch reads the tail from cow_src[s] and writes the whole
+ *                  block, this layer, every kv head, K and V, to the tail
+ *                  block with the new token in place -- what pkv_block_copy
+ *                  of (cow_src[s], tail) for this layer followed by
+ *                  pkv_kv_append would leave.  -1: no copy.  Read, like
+ *                  seq_lens and the tables, before the wait on the previous
+ *                  kernel.
  *   other arguments as pkv_paged_decode_attention.
  *
  * Result: the pools hold exactly what pkv_kv_append with that slot mapping
@@ -340,6 +357,7 @@ int pkv_paged_decode_attention(const pkv_cache_t* cache, int layer,
  */
 int pkv_append_paged_decode_attention(const pkv_cache_t* cache, int layer,
                                       const void* k_new, const void* v_new,
+                                      const int32_t* cow_src,
                                       const void* q, int num_seqs, int num_q_heads,
                                       const int32_t* block_tables, int max_blocks_per_seq,
                                       const int32_t* seq_lens, float scale, void* out,

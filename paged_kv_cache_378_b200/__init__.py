@@ -219,11 +219,12 @@ class BlockState:
                              self.free_state.data_ptr())
 
 
-def block_manager_step(state, block_size, order=None, stream=None):
+def block_manager_step(state, block_size, order=None, stream=None, with_cow_src=False):
     """One decode step of the block manager on the device (every sequence
     appends one token; ``order`` int32 ``[N]`` is the writer order).  Updates
     ``state`` in place; returns ``(slot_mapping int64 [N], copy_pairs int32
-    [N, 2], num_pairs int32 [1])`` on the device."""
+    [N, 2], num_pairs int32 [1])`` on the device, plus ``cow_src int32 [N]``
+    (each sequence's copy source, -1 if none) with ``with_cow_src``."""
     dev = state.block_tables.device
     N, maxb = state.block_tables.shape
     nb = state.refcount.shape[0]
@@ -234,11 +235,14 @@ def block_manager_step(state, block_size, order=None, stream=None):
     slots = torch.empty(N, dtype=torch.int64, device=dev)
     pairs = torch.empty((max(N, 1), 2), dtype=torch.int32, device=dev)
     npairs = torch.zeros(1, dtype=torch.int32, device=dev)
+    cow = torch.empty(max(N, 1), dtype=torch.int32, device=dev)
     c = state._c()
     rc = library().pkv_block_manager_step(
         ctypes.byref(c), N, maxb, nb, int(block_size), order.data_ptr() if order is not None else None,
-        slots.data_ptr(), pairs.data_ptr(), npairs.data_ptr(), _stream(dev, stream))
+        slots.data_ptr(), pairs.data_ptr(), npairs.data_ptr(), cow.data_ptr(), _stream(dev, stream))
     _check(rc, "block_manager_step")
+    if with_cow_src:
+        return slots, pairs[:N], npairs, cow[:N]
     return slots, pairs[:N], npairs
 
 
@@ -304,12 +308,14 @@ def paged_decode_attention(q, k_pool, v_pool, block_tables, seq_lens, block_size
 
 def append_paged_decode_attention(k_new, v_new, q, k_pool, v_pool, block_tables, seq_lens,
                                   block_size, scale, out, layer=0, workspace=None,
-                                  partition_tokens=0, stream=None):
+                                  partition_tokens=0, cow_src=None, stream=None):
     """Fused decode step of one layer: store each sequence's newest token
     (``k_new``/``v_new`` bf16 ``[N, H_kv, d]``, position ``seq_lens[s] - 1``,
     slot from the block table) and attend over the updated cache; writes
     ``out``.  Same result as ``kv_append`` with that slot mapping followed by
-    ``paged_decode_attention``."""
+    ``paged_decode_attention``.  ``cow_src`` (int32 ``[N]``, -1 = none): the
+    tail block of sequence s is made here as a copy of block ``cow_src[s]``
+    (this layer), as ``block_copy`` would before the append."""
     cache, (L, NB, H, B, D) = _cache(k_pool, v_pool)
     if int(block_size) != B:
         raise ValueError(f"block_size {block_size} does not match the pools ({B})")
@@ -332,8 +338,14 @@ def append_paged_decode_attention(k_new, v_new, q, k_pool, v_pool, block_tables,
     if workspace is not None:
         _need(workspace, "workspace", torch.uint8, dev)
         ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+    cow_ptr = None
+    if cow_src is not None:
+        _need(cow_src, "cow_src", torch.int32, dev)
+        if cow_src.shape != (N,):
+            raise ValueError("cow_src must be [N]")
+        cow_ptr = cow_src.data_ptr()
     rc = library().pkv_append_paged_decode_attention(
-        ctypes.byref(cache), int(layer), k_new.data_ptr(), v_new.data_ptr(), q.data_ptr(), N, Hq,
+        ctypes.byref(cache), int(layer), k_new.data_ptr(), v_new.data_ptr(), cow_ptr, q.data_ptr(), N, Hq,
         block_tables.data_ptr(), maxb, seq_lens.data_ptr(), float(scale), out.data_ptr(), ws_ptr,
         ws_bytes, int(partition_tokens), _stream(dev, stream))
     _check(rc, "append_paged_decode_attention")

@@ -47,7 +47,8 @@ SIGNATURES = {
         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "pkv_block_manager_step": (ctypes.c_int, [
         ctypes.POINTER(PkvBlockState), ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_void_p]),
     "pkv_attention_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 7),
     "pkv_partition_tokens": (ctypes.c_int, [ctypes.c_int] * 6),
     "pkv_workspace_init": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
@@ -57,6 +58,7 @@ SIGNATURES = {
         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]),
     "pkv_append_paged_decode_attention": (ctypes.c_int, [
         ctypes.POINTER(PkvCache), ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_void_p,
         ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_float,
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]),
     "pkv_paged_decode_attention_noalloc": (ctypes.c_int, [

@@ -73,6 +73,10 @@ struct AttnArgs {
     const uint4* v_new;
     uint16_t* k_pool;              // pool bases (all layers)
     uint16_t* v_pool;
+    // fused copy-on-write (with the fused append; may be null): sequence s's
+    // tail block is a fresh copy of block cow_src[s] (>= 0), made here for
+    // this layer: the tile reads the source and writes the copy
+    const int32_t* cow_src;        // [N]
     int cap_tiles;                 // > 0: no range longer than this many tiles
     int K;                         // warps in the grid
 };
@@ -104,7 +108,9 @@ struct AttnCfg {
     static constexpr int BAR_OFF = META_OFF + NW * STAGES * META_BYTES;
     // fused append: per stage, the new token's physical block (16-byte
     // header) and its K and V rows, brought by bulk copies with the tile
-    static constexpr int NEW_BYTES = 16 + 4 * D;
+    // header: new-row destinations (K, V), copy-on-write block destinations (K, V)
+    static constexpr int NEW_HDR = 32;
+    static constexpr int NEW_BYTES = NEW_HDR + 4 * D;
     static constexpr int NEW_OFF = BAR_OFF + NW * STAGES * 8;
     static constexpr int PREFIX_OFF = NEW_OFF + NW * STAGES * NEW_BYTES;
     static constexpr int SMEM_BYTES = PREFIX_OFF + (PREFIX_SMEM + 1) * 4 + 1024;   // + alignment slack
@@ -258,18 +264,6 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (pre_smem) s_prefix[0] = 0;
         else a.prefix_g[0] = 0;
     }
-    // Planning read only the lengths, which no kernel of this library writes;
-    // from here on the pool and the outputs are touched, so the kernel before
-    // this one on the stream must have finished.
-    pdl_wait();
-    if (blockIdx.x == 0) {                                // nothing to attend to: zero output
-        for (int s = tid; s < N; s += NT) {
-            if (clamp_len(__ldg(a.seq_lens + s), cap) == 0) {
-                uint4* o4 = reinterpret_cast<uint4*>(a.out + (size_t)s * Hq * D);
-                for (int c = 0; c < Hq * D / 8; ++c) o4[c] = make_uint4(0, 0, 0, 0);
-            }
-        }
-    }
     const long long K = a.K;
     Sched sc;
     sc.T = T;
@@ -312,6 +306,7 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
     long long r = r_first;                                // range of the next tile to issue
     long long f = 0, f_end = 0, f_stop = 0;
     int ps = 0, ph = 0, pt = 0, plen = 0, pnt = 0, next_len = 0;
+    int pcow = -1, next_cow = -1;                         // copy-on-write source of ps, ps + 1
     bool range_first = true;
     int ids = -1, ids_seq = -1, ids_base = 0;
     int pre = -1, pre_seq = -1, pre_base = 0;
@@ -324,19 +319,43 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (s >= N) return 0;
         return lens_smem ? s_len[s] : clamp_len(__ldg(a.seq_lens + s), cap);
     };
+    auto cow_of = [&](int s) -> int { return (a.cow_src && s < N) ? __ldg(a.cow_src + s) : -1; };
     auto advance_unit = [&]() {
         pt = 0;
         if (++ph < Hkv) return;
         ph = 0;
         ++ps;
         plen = next_len;
+        pcow = next_cow;
         pnt = (plen + TILE - 1) / TILE;
         while (pnt == 0 && ps + 1 < N) {   // skip empty sequences (rare, synchronous)
             ++ps;
             plen = seq_len(ps);
+            pcow = cow_of(ps);
             pnt = (plen + TILE - 1) / TILE;
         }
         next_len = seq_len(ps + 1);
+        next_cow = cow_of(ps + 1);
+    };
+    // Block ids of the current tile's batch of 32 logical blocks (one per
+    // lane), taken from the prefetched batch when it holds them; then the
+    // batch needed after this one is prefetched: the rest of this table row,
+    // else the row's start again for the next kv head, else the next
+    // sequence's row.
+    auto fetch_ids = [&](int lb0) {
+        if (ids_seq == ps && lb0 >= ids_base && lb0 + C::BPT <= ids_base + 32) return;
+        if (pre_seq == ps && lb0 >= pre_base && lb0 + C::BPT <= pre_base + 32) {
+            ids = pre; ids_seq = pre_seq; ids_base = pre_base;
+        } else {
+            ids = load_batch(ps, lb0, plen); ids_seq = ps; ids_base = lb0;
+        }
+        if ((ids_base + 32) * BS < plen) {
+            pre_seq = ps; pre_base = ids_base + 32; pre = load_batch(ps, pre_base, plen);
+        } else if (ph + 1 < Hkv && ids_base != 0) {
+            pre_seq = ps; pre_base = 0; pre = load_batch(ps, 0, plen);
+        } else if (ps + 1 < N) {
+            pre_seq = ps + 1; pre_base = 0; pre = load_batch(ps + 1, 0, next_len);
+        }
     };
     const bool have_work = r_first < r_stop;
     if (have_work) {
@@ -347,6 +366,23 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         plen = seq_len(ps);
         pnt = (plen + TILE - 1) / TILE;
         next_len = seq_len(ps + 1);
+        pcow = cow_of(ps);
+        next_cow = cow_of(ps + 1);
+        fetch_ids(pt * C::BPT);                           // the first tile's block ids
+    }
+
+    // Everything so far read only the lengths and the block tables, which no
+    // kernel of this library writes; from here on the pools, q and the
+    // outputs are touched, so the kernel before this one on the stream must
+    // have finished.
+    pdl_wait();
+    if (blockIdx.x == 0) {                                // nothing to attend to: zero output
+        for (int s = tid; s < N; s += NT) {
+            if (clamp_len(__ldg(a.seq_lens + s), cap) == 0) {
+                uint4* o4 = reinterpret_cast<uint4*>(a.out + (size_t)s * Hq * D);
+                for (int c = 0; c < Hq * D / 8; ++c) o4[c] = make_uint4(0, 0, 0, 0);
+            }
+        }
     }
 
     // Stage the next tile into stage `st`; false when this warp has no more tiles.
@@ -365,23 +401,7 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (f + 1 == f_end || pt == pnt - 1) flags |= F_LAST;
         range_first = false;
         const int lb0 = pt * C::BPT;
-        if (ids_seq != ps || lb0 < ids_base || lb0 + C::BPT > ids_base + 32) {
-            if (pre_seq == ps && lb0 >= pre_base && lb0 + C::BPT <= pre_base + 32) {
-                ids = pre; ids_seq = pre_seq; ids_base = pre_base;
-            } else {
-                ids = load_batch(ps, lb0, plen); ids_seq = ps; ids_base = lb0;
-            }
-            // prefetch the batch needed after this one: the rest of this table
-            // row, else the row's start again for the next kv head, else the
-            // next sequence's row
-            if ((ids_base + 32) * BS < plen) {
-                pre_seq = ps; pre_base = ids_base + 32; pre = load_batch(ps, pre_base, plen);
-            } else if (ph + 1 < Hkv && ids_base != 0) {
-                pre_seq = ps; pre_base = 0; pre = load_batch(ps, 0, plen);
-            } else if (ps + 1 < N) {
-                pre_seq = ps + 1; pre_base = 0; pre = load_batch(ps + 1, 0, next_len);
-            }
-        }
+        fetch_ids(lb0);
         int bid[C::BPT];
 #pragma unroll
         for (int j = 0; j < C::BPT; ++j) bid[j] = __shfl_sync(FULL, ids, lb0 - ids_base + j);
@@ -392,18 +412,29 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
             m.s = ps; m.h = ph; m.t = pt; m.len = plen; m.f = f; m.flags = flags; m.r = (int)r;
             meta[st] = m;
             if (fused_append && (flags & F_UNIT_END)) {
-                // where the new token's K and V rows go (null: block id out of range)
+                // where the new token's K and V rows go, and (copy-on-write) the
+                // copied tail block's rows of this head (null: none, or an id
+                // out of range)
                 uint16_t* dk = nullptr;
                 uint16_t* dv = nullptr;
+                uint16_t* ck = nullptr;
+                uint16_t* cv = nullptr;
                 if (nblk >= 0 && nblk < a.num_blocks) {
-                    const size_t prow =
-                        (size_t)(a.row_base + ((long long)nblk * Hkv + ph) * BS + (plen - 1) % BS);
-                    dk = a.k_pool + prow * D;
-                    dv = a.v_pool + prow * D;
+                    const size_t brow = (size_t)(a.row_base + ((long long)nblk * Hkv + ph) * BS);
+                    dk = a.k_pool + (brow + (plen - 1) % BS) * D;
+                    dv = a.v_pool + (brow + (plen - 1) % BS) * D;
+                    if (pcow >= 0 && pcow < a.num_blocks) {
+                        ck = a.k_pool + brow * D;
+                        cv = a.v_pool + brow * D;
+                    } else if (pcow >= a.num_blocks) {
+                        raise_status(PKV_DEV_RANGE);
+                    }
                 }
                 uint16_t** hdr = reinterpret_cast<uint16_t**>(newrows + (size_t)st * C::NEW_BYTES);
                 hdr[0] = dk;
                 hdr[1] = dv;
+                hdr[2] = ck;
+                hdr[3] = cv;
             }
             const uint32_t bar = smem_addr(&bars[st]);
             const uint32_t dK = smem_addr(ring + (size_t)st * C::STAGE_BYTES);
@@ -428,14 +459,17 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (app) {
                 unsigned char* nb = newrows + (size_t)st * C::NEW_BYTES;
                 const size_t row = ((size_t)ps * Hkv + ph) * CH;       // in 16-byte chunks
-                bulk_g2s(smem_addr(nb + 16), a.k_new + row, 2u * D, bar, pol_stream);
-                bulk_g2s(smem_addr(nb + 16 + 2 * D), a.v_new + row, 2u * D, bar, pol_stream);
+                bulk_g2s(smem_addr(nb + C::NEW_HDR), a.k_new + row, 2u * D, bar, pol_stream);
+                bulk_g2s(smem_addr(nb + C::NEW_HDR + 2 * D), a.v_new + row, 2u * D, bar, pol_stream);
             }
 #pragma unroll
             for (int j = 0; j < C::BPT; ++j) {
                 if (j * BS >= nv || bid[j] < 0 || bid[j] >= a.num_blocks) continue;
+                // copy-on-write: the tail block is read from its source
+                const int blk = (app && pcow >= 0 && pcow < a.num_blocks &&
+                                 lb0 + j == (plen - 1) / BS) ? pcow : bid[j];
                 // pool row of (layer, block, head, row 0); the layer is in row_base
-                const int y = (int)(a.row_base + ((long long)bid[j] * Hkv + ph) * BS);
+                const int y = (int)(a.row_base + ((long long)blk * Hkv + ph) * BS);
                 const uint32_t off = (uint32_t)(j * TS::RPB * 128);
 #pragma unroll
                 for (int hf = 0; hf < TS::HALVES; ++hf) {
@@ -653,13 +687,30 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const int c = lane % CH;
                 uint4* dst = reinterpret_cast<uint4* const*>(nb)[lane < CH ? 0 : 1];
                 if (dst) {
-                    const uint4 v = reinterpret_cast<const uint4*>(nb + 16)[lane];   // K row, then V row
+                    const uint4 v = reinterpret_cast<const uint4*>(nb + C::NEW_HDR)[lane];   // K row, then V row
                     *reinterpret_cast<uint4*>(sKp + (lane < CH ? 0 : C::KT_BYTES) +
                                               TS::offset(m.len - 1 - m.t * TILE, c)) = v;
                     dst[c] = v;
                 }
             }
             __syncwarp();
+            // Copy-on-write: the tail block came from its source; with the new
+            // row in place, all of its rows (this head, this layer, K and V)
+            // go to the fresh block, before V rows past the length are zeroed.
+            uint4* ck = reinterpret_cast<uint4* const*>(nb)[2];
+            if (ck) {
+                uint4* cv = reinterpret_cast<uint4* const*>(nb)[3];
+                const int t0 = ((m.len - 1) / BS) * BS - m.t * TILE;   // tail block's first token in the tile
+                for (int e = lane; e < 2 * BS * CH; e += 32) {
+                    const int kv = e / (BS * CH);
+                    const int rc = e - kv * BS * CH;
+                    const int row = rc / CH, c = rc - row * CH;
+                    const uint4 v = *reinterpret_cast<const uint4*>(sKp + (kv ? C::KT_BYTES : 0) +
+                                                                    TS::offset(t0 + row, c));
+                    (kv ? cv : ck)[row * CH + c] = v;
+                }
+                __syncwarp();                                 // before V rows are zeroed
+            }
         }
         if (m.flags & F_FIRST) {
             load_q_frags<D, G>(qa, reinterpret_cast<const uint16_t*>(qslots + (size_t)st * C::Q_BYTES),

@@ -37,6 +37,7 @@ struct BmArgs {
     int64_t* slot_mapping;      // [N] out, by sequence
     int32_t* copy_pairs;        // [N][2] out, (src, dst) in writer order
     int32_t* num_pairs;         // [1] out
+    int32_t* cow_src;           // [N] out (may be null): copy source per sequence, -1 if none
     int num_seqs;
     int max_blocks;
     int num_blocks;
@@ -160,6 +161,7 @@ __global__ void __launch_bounds__(BM_THREADS, 1) block_manager_kernel(const BmAr
             }
             *entry = nb;
         }
+        if (a.cow_src) a.cow_src[s] = copies[k] ? s_tail[k * BM_THREADS + tid] : -1;
         a.slot_mapping[s] = (int64_t)(*entry) * B + p % B;
         a.seq_lens[s] = p + 1;
     }

@@ -301,7 +301,8 @@ unsigned char* noalloc_scratch_ptr() {
 // Shared body of the attention entry points that take a workspace; k_new and
 // v_new non-null = fused append of each sequence's newest token.
 int attention_with_workspace(const pkv_cache_t* cache, int layer, const void* k_new,
-                                    const void* v_new, const void* q, int num_seqs, int num_q_heads,
+                                    const void* v_new, const int32_t* cow_src, const void* q,
+                                    int num_seqs, int num_q_heads,
                                     const int32_t* block_tables, int max_blocks_per_seq,
                                     const int32_t* seq_lens, float scale, void* out, void* workspace,
                                     size_t workspace_bytes, int partition_tokens, void* stream) {
@@ -352,6 +353,7 @@ int attention_with_workspace(const pkv_cache_t* cache, int layer, const void* k_
     a.R_max = w.R_max;
     a.k_new = static_cast<const uint4*>(k_new);
     a.v_new = static_cast<const uint4*>(v_new);
+    a.cow_src = k_new ? cow_src : nullptr;
     a.k_pool = static_cast<uint16_t*>(cache->k_pool);
     a.v_pool = static_cast<uint16_t*>(cache->v_pool);
     a.cap_tiles = w.cap_tiles;
@@ -503,7 +505,7 @@ int pkv_prefix_block_hashes(const int32_t* tokens, int max_tokens, const int32_t
 int pkv_block_manager_step(const pkv_block_state_t* st, int num_seqs, int max_blocks_per_seq,
                            int num_blocks, int block_size, const int32_t* order,
                            int64_t* slot_mapping, int32_t* copy_pairs, int32_t* num_pairs,
-                           void* stream) {
+                           int32_t* cow_src, void* stream) {
     if (!st) return PKV_ERR_NULL;
     if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || block_size <= 0)
         return PKV_ERR_SHAPE;
@@ -522,6 +524,7 @@ int pkv_block_manager_step(const pkv_block_state_t* st, int num_seqs, int max_bl
     a.slot_mapping = slot_mapping;
     a.copy_pairs = copy_pairs;
     a.num_pairs = num_pairs;
+    a.cow_src = cow_src;
     a.num_seqs = num_seqs;
     a.max_blocks = max_blocks_per_seq;
     a.num_blocks = num_blocks;
@@ -559,19 +562,20 @@ int pkv_paged_decode_attention(const pkv_cache_t* cache, int layer, const void* 
                                int num_q_heads, const int32_t* block_tables, int max_blocks_per_seq,
                                const int32_t* seq_lens, float scale, void* out, void* workspace,
                                size_t workspace_bytes, int partition_tokens, void* stream) {
-    return attention_with_workspace(cache, layer, nullptr, nullptr, q, num_seqs, num_q_heads,
+    return attention_with_workspace(cache, layer, nullptr, nullptr, nullptr, q, num_seqs, num_q_heads,
                                     block_tables, max_blocks_per_seq, seq_lens, scale, out, workspace,
                                     workspace_bytes, partition_tokens, stream);
 }
 
 int pkv_append_paged_decode_attention(const pkv_cache_t* cache, int layer, const void* k_new,
-                                      const void* v_new, const void* q, int num_seqs,
+                                      const void* v_new, const int32_t* cow_src, const void* q,
+                                      int num_seqs,
                                       int num_q_heads, const int32_t* block_tables,
                                       int max_blocks_per_seq, const int32_t* seq_lens, float scale,
                                       void* out, void* workspace, size_t workspace_bytes,
                                       int partition_tokens, void* stream) {
     if (!k_new || !v_new) return PKV_ERR_NULL;
-    return attention_with_workspace(cache, layer, k_new, v_new, q, num_seqs, num_q_heads,
+    return attention_with_workspace(cache, layer, k_new, v_new, cow_src, q, num_seqs, num_q_heads,
                                     block_tables, max_blocks_per_seq, seq_lens, scale, out, workspace,
                                     workspace_bytes, partition_tokens, stream);
 }
@@ -628,6 +632,7 @@ int pkv_paged_decode_attention_noalloc(const pkv_cache_t* cache, int layer, cons
     a.prefix_g = reinterpret_cast<long long*>(ws + w.prefix_off);
     a.k_new = nullptr;                                // no fused append here
     a.v_new = nullptr;
+    a.cow_src = nullptr;
     a.k_pool = static_cast<uint16_t*>(cache->k_pool);
     a.v_pool = static_cast<uint16_t*>(cache->v_pool);
     a.R_max = w.R_max;

@@ -37,12 +37,22 @@ def device_inputs(w, device="cuda"):
     )
 
 
-def gpu_step(pkv, w, dev_in, layers=None, partition_tokens=None, workspace=None, fused=False):
+def cow_sources(w):
+    """Per sequence, the source block of this step's copy-on-write (-1 if
+    none): the pair whose destination is the sequence's tail block."""
+    src_of = {int(d): int(s) for s, d in w.copy_pairs}
+    tails = w.block_tables[np.arange(w.num_seqs), (w.seq_lens.astype(np.int64) - 1) // w.block_size]
+    return np.array([src_of.get(int(t), -1) for t in tails], np.int32)
+
+
+def gpu_step(pkv, w, dev_in, layers=None, partition_tokens=None, workspace=None, fused=False,
+             cow=False):
     """Run the step with the CUDA library; returns {layer: out bf16 tensor}.
 
     ``fused``: append and attention of each layer in one call
     (``append_paged_decode_attention``) instead of ``kv_append`` then
-    ``paged_decode_attention``."""
+    ``paged_decode_attention``.  ``cow`` (with ``fused``): the copy-on-write is
+    folded into those calls too (``cow_src``) instead of a ``block_copy``."""
     spec = w.spec
     part = spec.partition_tokens if partition_tokens is None else partition_tokens
     L = dev_in["k_pool"].shape[0]
@@ -51,7 +61,11 @@ def gpu_step(pkv, w, dev_in, layers=None, partition_tokens=None, workspace=None,
         workspace = pkv.make_workspace(w.num_seqs, spec.num_q_heads, spec.num_kv_heads,
                                        spec.head_dim, w.max_blocks, w.block_size, part,
                                        device=dev_in["q"].device)
-    pkv.block_copy(dev_in["pairs"], dev_in["k_pool"], dev_in["v_pool"])
+    cow_src = None
+    if fused and cow:
+        cow_src = torch.from_numpy(cow_sources(w)).to(dev_in["q"].device)
+    else:
+        pkv.block_copy(dev_in["pairs"], dev_in["k_pool"], dev_in["v_pool"])
     outs = {}
     for layer in layers:
         out = torch.empty_like(dev_in["q"][layer])
@@ -59,7 +73,8 @@ def gpu_step(pkv, w, dev_in, layers=None, partition_tokens=None, workspace=None,
             pkv.append_paged_decode_attention(
                 dev_in["k_new"][layer], dev_in["v_new"][layer], dev_in["q"][layer],
                 dev_in["k_pool"], dev_in["v_pool"], dev_in["tables"], dev_in["lens"], w.block_size,
-                spec.scale, out, layer=layer, workspace=workspace, partition_tokens=part)
+                spec.scale, out, layer=layer, workspace=workspace, partition_tokens=part,
+                cow_src=cow_src)
             outs[layer] = out
             continue
         pkv.kv_append(dev_in["k_new"][layer], dev_in["v_new"][layer], dev_in["slots"],

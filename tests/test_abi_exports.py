@@ -87,11 +87,11 @@ def test_host_argument_checks_before_launch():
     assert att(P(c), 0, 16, 2, 8, 16, 4096, 16, 0.125, 16, 256, need - 1, 512, None) == -4
     # fused append + attention: both new-row pointers required and aligned
     fa = lib.pkv_append_paged_decode_attention
-    assert fa(P(c), 0, None, 16, 16, 2, 8, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -1
-    assert fa(P(c), 0, 16, None, 16, 2, 8, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -1
-    assert fa(P(c), 0, 24, 16, 16, 2, 8, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -3
-    assert fa(P(c), 0, 16, 16, 16, 2, 6, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -5
-    assert fa(P(c), 0, 16, 16, 16, 0, 8, 16, 4, 16, 0.125, 16, None, 0, 0, None) == 0
+    assert fa(P(c), 0, None, 16, None, 16, 2, 8, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -1
+    assert fa(P(c), 0, 16, None, None, 16, 2, 8, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -1
+    assert fa(P(c), 0, 24, 16, None, 16, 2, 8, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -3
+    assert fa(P(c), 0, 16, 16, None, 16, 2, 6, 16, 4, 16, 0.125, 16, 256, need, 512, None) == -5
+    assert fa(P(c), 0, 16, 16, None, 16, 0, 8, 16, 4, 16, 0.125, 16, None, 0, 0, None) == 0
     # block copy with a device-side count: the count pointer is required
     assert lib.pkv_block_copy_device_count(P(c), 16, 4, None, None) == -1
     assert lib.pkv_block_copy_device_count(P(c), 16, 0, None, None) == 0
@@ -107,13 +107,13 @@ def test_host_argument_checks_before_launch():
     # device block manager step: state required, sizes checked, at most 4096 sequences
     st = _lib.PkvBlockState(16, 16, 16, 16, 16)
     bm = lib.pkv_block_manager_step
-    assert bm(None, 4, 8, 64, 16, None, 16, 16, 16, None) == -1
-    assert bm(P(st), -1, 8, 64, 16, None, 16, 16, 16, None) == -2
-    assert bm(P(st), 4, 0, 64, 16, None, 16, 16, 16, None) == -2
-    assert bm(P(st), 4097, 8, 64, 16, None, 16, 16, 16, None) == -5
-    assert bm(P(st), 0, 8, 64, 16, None, 16, 16, 16, None) == 0
-    assert bm(P(st), 4, 8, 64, 16, None, None, 16, 16, None) == -1
-    assert bm(P(_lib.PkvBlockState(16, 0, 16, 16, 16)), 4, 8, 64, 16, None, 16, 16, 16, None) == -1
+    assert bm(None, 4, 8, 64, 16, None, 16, 16, 16, None, None) == -1
+    assert bm(P(st), -1, 8, 64, 16, None, 16, 16, 16, None, None) == -2
+    assert bm(P(st), 4, 0, 64, 16, None, 16, 16, 16, None, None) == -2
+    assert bm(P(st), 4097, 8, 64, 16, None, 16, 16, 16, None, None) == -5
+    assert bm(P(st), 0, 8, 64, 16, None, 16, 16, 16, None, None) == 0
+    assert bm(P(st), 4, 8, 64, 16, None, None, 16, 16, None, None) == -1
+    assert bm(P(_lib.PkvBlockState(16, 0, 16, 16, 16)), 4, 8, 64, 16, None, 16, 16, 16, None, None) == -1
 
 
 def test_workspace_and_partition_sizes():

@@ -211,3 +211,48 @@ def test_workload_steps_at_full_size(key, B):
     for s in range(w.num_seqs):
         nb = -(-int(w.seq_lens[s]) // w.block_size)
         assert np.array_equal(tab[s, :nb], w.block_tables[s, :nb])
+
+
+def test_device_step_with_copy_on_write_folded_into_attention():
+    # manager -> one fused launch that copies the shared tails, appends and
+    # attends: pools equal the oracle's block copy + append, output within
+    # tolerance of the oracle
+    from oracle import attention as oa
+    from .stepping import assert_close, f64, u16
+    rng = np.random.default_rng(11)
+    B, H, D, G, NB = 16, 2, 64, 4, 120
+    bm = BlockManager(NB, B, free_order=rng.permutation(NB))
+    bm.add_sequence(0, 45)
+    for c in range(1, 5):
+        bm.fork(0, c)
+    for s in range(5, 12):
+        bm.add_sequence(s, int(rng.integers(1, 90)))
+    writers = list(range(12))
+    st = _snapshot(bm, writers, 8)
+    g = torch.Generator().manual_seed(11)
+    kp = torch.randn((1, NB, H, B, D), generator=g).to(torch.bfloat16)
+    vp = torch.randn((1, NB, H, B, D), generator=g).to(torch.bfloat16)
+    q = torch.randn((12, H * G, D), generator=g).to(torch.bfloat16)
+    kn = torch.randn((12, H, D), generator=g).to(torch.bfloat16)
+    vn = torch.randn((12, H, D), generator=g).to(torch.bfloat16)
+    kd, vd = kp.cuda(), vp.cuda()
+    slots, pairs, npairs, cow = pkv.block_manager_step(st, B, with_cow_src=True)
+    out = torch.empty_like(q).cuda()
+    ws = pkv.make_workspace(12, H * G, H, D, 8, B, 0)
+    pkv.append_paged_decode_attention(kn.cuda(), vn.cuda(), q.cuda(), kd, vd, st.block_tables,
+                                      st.seq_lens, B, D ** -0.5, out, workspace=ws, cow_src=cow)
+    torch.cuda.synchronize()
+    assert pkv.get_device_status(reset=True) == 0
+    want_slots = [bm.append_slot(s) for s in writers]
+    want_pairs = np.array(bm.take_copy_pairs(), np.int32).reshape(-1, 2)
+    assert len(want_pairs) == 4 and int(npairs.item()) == 4
+    assert slots.cpu().tolist() == want_slots
+    ek, ev = oa.block_copy(u16(kp), u16(vp), want_pairs)
+    ek, ev = oa.kv_append(ek[0], ev[0], u16(kn), u16(vn), np.array(want_slots), B)
+    assert np.array_equal(u16(kd[0]), ek) and np.array_equal(u16(vd[0]), ev)
+    tables = np.full((12, 8), -1, np.int32)
+    for s in writers:
+        tables[s, :len(bm.tables[s])] = bm.tables[s]
+    lens = np.array([bm.lengths[s] for s in writers], np.int32)
+    ref = oa.paged_decode_attention(u16(q), ek, ev, tables, lens, B, D ** -0.5)
+    assert_close(f64(out), ref, "copy-on-write folded into attention")

@@ -32,10 +32,11 @@ def _clean_status():
     yield
 
 
-def _fused_vs_oracle_and_two_call(w, partition=None, layers=None):
+def _fused_vs_oracle_and_two_call(w, partition=None, layers=None, cow=False):
     dev_f = device_inputs(w)
     dev_t = device_inputs(w)
-    outs_f = gpu_step(pkv, w, dev_f, layers=layers, partition_tokens=partition, fused=True)
+    outs_f = gpu_step(pkv, w, dev_f, layers=layers, partition_tokens=partition, fused=True,
+                      cow=cow)
     outs_t = gpu_step(pkv, w, dev_t, layers=layers, partition_tokens=partition)
     assert pkv.get_device_status(reset=True) == 0
     for l, out in outs_f.items():
@@ -52,6 +53,26 @@ def _fused_vs_oracle_and_two_call(w, partition=None, layers=None):
 @pytest.mark.parametrize("key", ["tiny", "llama1b_layer", "continuous_batch"])
 def test_fused_step_matches_oracle(key):
     _fused_vs_oracle_and_two_call(make_workload(key))
+
+
+@pytest.mark.parametrize("partition", [0, 64])
+def test_fused_copy_on_write_continuous_batch(partition):
+    # 28 copy-on-write pairs folded into the attention launch: the copied tails
+    # (every head, K and V, NaN-poisoned destinations) must come out bit exact
+    w = make_workload("continuous_batch")
+    assert len(w.copy_pairs) > 0
+    _fused_vs_oracle_and_two_call(w, partition=partition, cow=True)
+
+
+@pytest.mark.parametrize("D,G,B", [(64, 4, 16), (128, 4, 16), (64, 8, 4), (128, 1, 32), (64, 2, 8)])
+def test_fused_copy_on_write_shapes(D, G, B):
+    spec = WorkloadSpec(key="custom", title="custom", num_layers=2, num_seqs=20,
+                        num_q_heads=2 * G, num_kv_heads=2, head_dim=D, block_size=B,
+                        seed=500 + D + G + B, lengths="uniform:1,200", shared_groups=2,
+                        shared_group_size=4, shared_prefix=3 * B)
+    w = make_workload(spec)
+    assert len(w.copy_pairs) > 0
+    _fused_vs_oracle_and_two_call(w, partition=0, cow=True)
 
 
 @pytest.mark.parametrize("partition", [512, 0])
