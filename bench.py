@@ -736,7 +736,8 @@ def main():
     nl = spec.num_layers
     for i in range(args.steps):
         j = i // EVENT_EVERY
-        gs.run(i, evs[j * nl:(j + 1) * nl] if i % EVENT_EVERY == 0 else None)
+        bracket = not only_attention and i % EVENT_EVERY == 0
+        gs.run(i, evs[j * nl:(j + 1) * nl] if bracket else None)
     t_end.record(gs.stream)
     torch.cuda.synchronize(device)
     wall1 = time.time()
