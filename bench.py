@@ -54,10 +54,16 @@ KERNEL_SOURCES = ["pkv_device.cuh", "attn_common.cuh", "attn_paged.cuh"]
 # ---------------------------------------------------------------------------
 
 def kernel_source_hash():
+    """Hash of the attention kernel's device sources with comments and blank
+    lines removed, so an edit to comments alone keeps a capture valid."""
+    import re
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "paged_kv_cache_378_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "paged_kv_cache_378_b200", "csrc", f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        lines = [ln.split("//", 1)[0].rstrip() for ln in text.splitlines()]
+        h.update("\n".join(ln for ln in lines if ln.strip()).encode())
     return h.hexdigest()[:16]
 
 

@@ -16,14 +16,20 @@
 // across unit and range boundaries, so it never drains between sequences,
 // and every warp gets the same number of tiles whatever the length mix.  A
 // unit inside one range is finished by its warp; a unit cut by range
-// boundaries leaves one partial per range, and the last range to finish (an
-// atomic ticket per unit, reset by that range) merges them in range order,
-// so the result does not depend on which piece finishes last.
+// boundaries leaves one partial per range.  Pieces count themselves on a
+// ticket; the last one merges them in range order into its own registers
+// (a piece that finds every other piece already counted merges without
+// publishing itself).  Units of more than 8 pieces merge in two levels:
+// groups of 8 ranges, then the groups.  The fold order is fixed, so the
+// result does not depend on which piece finishes last.
 //
 // Planning.  Every CTA reads the sequence lengths once and scans them into
 // a prefix of tiles per sequence, kept in shared memory (in global memory,
 // written identically by every CTA, for batches of more than PREFIX_SMEM
-// sequences); a warp finds its first tile by binary search.
+// sequences); a warp finds its first tile by binary search and loads its
+// first block ids.  All of this reads only the lengths and the tables and
+// runs before the wait on the previous kernel (programmatic dependent
+// launch); the rest of the kernel runs after it.
 //
 // Data movement.  Each warp owns a ring of STAGES shared-memory stages.  One
 // lane issues, per stage, TMA tensor loads (cp.async.bulk.tensor, 2-D tensor
@@ -33,6 +39,12 @@
 // ldmatrix reads of K and V conflict-free.  Rows of a tail block past the
 // sequence's length are loaded with the block but masked: their scores are
 // -inf and their V rows are zeroed in shared memory before the P V product.
+//
+// Fused append and copy-on-write (k_new set).  The unit's last tile also
+// brings the new token's K and V rows (bulk copies into a staging area); they
+// replace the stale row in shared memory and are stored in their slot.  With
+// cow_src, the tail block is fetched from its copy source and written whole
+// (this layer, this kv head, K and V, new row included) to the fresh block.
 //
 // Compute.  Tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with
 // the G query heads as the MMA rows; see attn_common.cuh.
