@@ -307,6 +307,23 @@ def packed_buffers(like, device, pin):
     return raw, views
 
 
+STEP_TEXT = {"cow": "per layer one launch: copy-on-write of shared tails, append of the new "
+                    "token, attention",
+             "fused": "block_copy, then per layer one fused append+attention launch",
+             "two-call": "block_copy, then per layer kv_append and attention launches"}
+
+
+def workload_config(pkv, key, spec, w, B, part, world, mode):
+    """The ``config`` object both arms print for a workload."""
+    return {"workload": key, "title": spec.title, "num_seqs": w.num_seqs,
+            "num_layers": spec.num_layers, "q_heads": spec.num_q_heads,
+            "kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim, "block_size": B,
+            "partition_tokens": pkv.partition_tokens(w.num_seqs, spec.num_kv_heads,
+                                                     spec.head_dim, w.max_blocks, B, part),
+            "parallelism": f"dp{world} (independent batches, no collective)",
+            "step": STEP_TEXT[mode]}
+
+
 def cow_sources(w):
     """Per sequence, the source block of this step's copy-on-write (-1 if
     none): the pair whose destination is the sequence's tail block."""
@@ -606,6 +623,12 @@ def run_reference(args):
     B = args.block_size or spec.block_size
     lim = limit_blas_threads()
     w, host = host_workload(args.workload, B, spec.seed)
+    # the same config object our arm prints (the library's partition rounding
+    # is host arithmetic; nothing runs on the GPU here)
+    import paged_kv_cache_378_b200 as pkv
+    part = spec.partition_tokens if args.partition < 0 else args.partition
+    ref_config = workload_config(pkv, args.workload, spec, w, B, part,
+                                 int(os.environ.get("WORLD_SIZE", "1")), args.step)
     kp, vp = oa.block_copy(host["k"], host["v"], w.copy_pairs)
     k2, v2 = oa.kv_append(kp[0], vp[0], host["k_new"][0], host["v_new"][0], w.slot_mapping,
                           w.block_size)
@@ -641,7 +664,7 @@ def run_reference(args):
             "n_gpus": int(os.environ.get("WORLD_SIZE", args.gpus)), "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "block_size": B},
+            "config": ref_config,
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -810,19 +833,9 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "title": spec.title, "num_seqs": w.num_seqs,
-                   "num_layers": spec.num_layers, "q_heads": spec.num_q_heads,
-                   "kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim, "block_size": B,
-                   "partition_tokens": pkv.partition_tokens(w.num_seqs, spec.num_kv_heads,
-                                                            spec.head_dim, w.max_blocks, B, part),
-                   "l2": f"inputs larger than L2: {nrep} rotating copies of the KV pools, "
-                         f"{nrep * pool_bytes / 1e9:.2f} GB vs {l2 / 1e6:.0f} MB L2",
-                   "parallelism": f"dp{world} (independent batches, no collective)",
-                   "step": {"cow": "per layer one launch: copy-on-write of shared tails, "
-                                   "append of the new token, attention",
-                            "fused": "block_copy, then per layer one fused append+attention launch",
-                            "two-call": "block_copy, then per layer kv_append and attention "
-                                        "launches"}[gs.mode]},
+        "config": dict(workload_config(pkv, args.workload, spec, w, B, part, world, gs.mode),
+                       l2=f"inputs larger than L2: {nrep} rotating copies of the KV pools, "
+                          f"{nrep * pool_bytes / 1e9:.2f} GB vs {l2 / 1e6:.0f} MB L2"),
         "pct_hbm_peak": 100.0 * value / peak,
         # one token per sequence per layer: N x L tokens cross a layer per step
         "decode_tokens_per_s_per_layer": seqs_total * spec.num_layers / (ms_per_step * 1e-3),

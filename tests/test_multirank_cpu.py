@@ -76,8 +76,12 @@ def test_reference_arm_on_non_zero_rank_does_nothing(monkeypatch, capsys):
 def test_reference_arm_prints_one_line(monkeypatch, capsys):
     import json
     monkeypatch.setenv("RANK", "0")
-    args = type("A", (), {"workload": "tiny", "block_size": 0, "steps": 3, "warmup": 3, "gpus": 1})
+    args = type("A", (), {"workload": "tiny", "block_size": 0, "steps": 3, "warmup": 3, "gpus": 1,
+                          "partition": -1, "step": "cow"})
     assert bench.run_reference(args) == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    # the same config object the GPU arm prints for this workload
+    assert line["config"]["workload"] == "tiny" and line["config"]["num_seqs"] == 4
+    assert line["config"]["step"] == bench.STEP_TEXT["cow"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
