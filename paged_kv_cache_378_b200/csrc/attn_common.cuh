@@ -65,13 +65,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // with the 128-byte swizzle, 64 dims (128 bytes) per row per half; a block
 // starts on a 1024-byte boundary (blocks of fewer than 8 rows are padded to
 // 8), so the 16-byte chunk c of smem row r sits at chunk c ^ (r & 7).
-#ifndef PKV_ATTN_D64_TILE
-#define PKV_ATTN_D64_TILE 32   // tokens per stage at head_dim 64 with blocks of 8 or 16
-#endif
-
 template <int D, int BS>
 struct TileSmem {
-    static constexpr int TILE = BS >= 32 ? BS : ((D == 64 && BS >= 8) ? PKV_ATTN_D64_TILE : 16);   // tokens per stage
+    static constexpr int TILE = BS >= 32 ? BS : ((D == 64 && BS >= 8) ? 32 : 16);   // tokens per stage
     static constexpr int BPT = TILE / BS;                // physical blocks per stage
     static constexpr int RPB = BS < 8 ? 8 : BS;          // smem rows per block
     static constexpr int TROWS = BPT * RPB;              // smem rows per tile

@@ -68,8 +68,7 @@ size_t layer_elems(const pkv_cache_t* c) {
 
 // tokens per pipeline stage of the attention kernel (TileSmem::TILE)
 int tile_tokens(int head_dim, int block_size) {
-    return block_size >= 32 ? block_size
-                            : ((head_dim == 64 && block_size >= 8) ? PKV_ATTN_D64_TILE : 16);
+    return block_size >= 32 ? block_size : ((head_dim == 64 && block_size >= 8) ? 32 : 16);
 }
 
 // Launch with programmatic stream serialization: the kernel may start while
