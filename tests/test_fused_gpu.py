@@ -115,3 +115,26 @@ def test_fused_binding_checks_new_row_shapes():
         pkv.append_paged_decode_attention(dev["k_new"][0][:-1], dev["v_new"][0], dev["q"][0],
                                           dev["k_pool"], dev["v_pool"], dev["tables"], dev["lens"],
                                           w.block_size, w.spec.scale, out)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_random_shapes_fuzz(seed):
+    # random head_dim, group, block size, batch, length mix, sharing and
+    # partition cap; the one-launch step (copy-on-write, append, attention)
+    # against the oracle and against the two-call path
+    rng = np.random.default_rng(1000 + seed)
+    D = int(rng.choice([64, 128]))
+    G = int(rng.choice([1, 2, 4, 8]))
+    B = int(rng.choice([4, 8, 16, 32]))
+    Hkv = int(rng.choice([1, 2, 4]))
+    N = int(rng.integers(9, 40))
+    hi = int(rng.choice([40, 300, 1500]))
+    groups = int(rng.integers(0, 3))
+    spec = WorkloadSpec(key="custom", title="custom", num_layers=int(rng.integers(1, 3)),
+                        num_seqs=N, num_q_heads=Hkv * G, num_kv_heads=Hkv, head_dim=D,
+                        block_size=B, seed=2000 + seed, lengths=f"uniform:1,{hi}",
+                        shared_groups=groups, shared_group_size=4 if groups else 0,
+                        shared_prefix=2 * B if groups else 0)
+    w = make_workload(spec)
+    part = int(rng.choice([0, 0, 32, 64, 256]))
+    _fused_vs_oracle_and_two_call(w, partition=part, cow=bool(groups))
