@@ -138,3 +138,15 @@ def test_random_shapes_fuzz(seed):
     w = make_workload(spec)
     part = int(rng.choice([0, 0, 32, 64, 256]))
     _fused_vs_oracle_and_two_call(w, partition=part, cow=bool(groups))
+
+
+@pytest.mark.parametrize("N", [800, 2500])
+def test_batches_past_the_shared_memory_prefix(N):
+    # more than 768 sequences: the tile prefix lives in the workspace and the
+    # lengths are read from global memory; with copy-on-write groups
+    spec = WorkloadSpec(key="custom", title="custom", num_layers=1, num_seqs=N, num_q_heads=4,
+                        num_kv_heads=1, head_dim=64, block_size=16, seed=3000 + N,
+                        lengths="uniform:1,70", shared_groups=3, shared_group_size=5,
+                        shared_prefix=32)
+    w = make_workload(spec)
+    _fused_vs_oracle_and_two_call(w, partition=0, cow=True)
