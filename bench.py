@@ -462,8 +462,8 @@ def prefix_hash_timing(pkv, w, device, iters=50):
         busy.zero_()
         if i >= 3:
             evs[i - 3][0].record(stream)
-        if lib.pkv_prefix_block_hashes(tok.data_ptr(), T, lens.data_ptr(), None, N, w.block_size,
-                                       out.data_ptr(), mb, sp):
+        if lib.pkv_prefix_block_hashes(tok.data_ptr(), T, lens.data_ptr(), None, None, None, N,
+                                       w.block_size, out.data_ptr(), mb, sp):
             raise SystemExit("prefix hash refused its arguments")
         if i >= 3:
             evs[i - 3][1].record(stream)

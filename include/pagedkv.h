@@ -188,13 +188,19 @@ int pkv_swap_blocks(const pkv_cache_t* device_cache, const pkv_cache_t* host_cac
  *   tokens       device int32 [num_seqs][max_tokens], token ids by position
  *   seq_lens     device int32 [num_seqs]; blocks 0 .. seq_lens/B - 1 are hashed
  *   extra_keys   device uint64 [num_seqs], or NULL for 0
- *   hashes       device uint64 [num_seqs][max_blocks] out; entries past a
- *                sequence's full blocks are not written
+ *   first_block  device int32 [num_seqs], or NULL for 0: hash only blocks
+ *                first_block[s] .. seq_lens/B - 1 (resuming, e.g. in decode
+ *                only the block that just became full)
+ *   parent_hashes device uint64 [num_seqs], or NULL: hash of block
+ *                first_block[s] - 1 (unused where first_block[s] is 0)
+ *   hashes       device uint64 [num_seqs][max_blocks] out; entries outside
+ *                [first_block, full blocks) are not written
  * A length above max_tokens, or more full blocks than max_blocks, sets
  * PKV_DEV_LENGTH and is clamped.
  */
 int pkv_prefix_block_hashes(const int32_t* tokens, int max_tokens, const int32_t* seq_lens,
-                            const uint64_t* extra_keys, int num_seqs, int block_size,
+                            const uint64_t* extra_keys, const int32_t* first_block,
+                            const uint64_t* parent_hashes, int num_seqs, int block_size,
                             uint64_t* hashes, int max_blocks, void* stream);
 
 /*

@@ -138,14 +138,17 @@ def block_copy(src_dst_pairs, k_pool, v_pool, num_pairs=None, stream=None):
 
 
 def prefix_block_hashes(tokens, seq_lens, block_size, extra_keys=None, max_blocks=None,
-                        stream=None):
+                        first_block=None, parent_hashes=None, out=None, stream=None):
     """Hash of every full block of every sequence (FNV-1a 64 chain over the
     parent hash, the block's tokens and the sequence's extra key).
 
     ``tokens`` int32 CUDA ``[N, T]``; ``seq_lens`` int32 ``[N]``; ``extra_keys``
     int64 ``[N]`` (bit patterns of uint64) or None.  Returns int64 ``[N,
-    max_blocks]`` holding the uint64 bit patterns; entries past a sequence's
-    full blocks are zero."""
+    max_blocks]`` holding the uint64 bit patterns.  ``first_block`` (int32
+    ``[N]``) and ``parent_hashes`` (int64 ``[N]``, the hash of block
+    first_block - 1) resume a sequence's chain, e.g. for only the block that
+    just became full; ``out`` receives the hashes in place (entries outside
+    the hashed blocks keep their values; a fresh output starts at zero)."""
     dev = tokens.device
     _need(tokens, "tokens", torch.int32, dev)
     _need(seq_lens, "seq_lens", torch.int32, dev)
@@ -157,11 +160,24 @@ def prefix_block_hashes(tokens, seq_lens, block_size, extra_keys=None, max_block
         if extra_keys.shape != (N,):
             raise ValueError("extra_keys must be [N]")
     mb = T // int(block_size) if max_blocks is None else int(max_blocks)
-    out = torch.zeros((N, max(mb, 1)), dtype=torch.int64, device=dev)
+    ptrs = []
+    for t, name, dt in ((first_block, "first_block", torch.int32),
+                        (parent_hashes, "parent_hashes", torch.int64)):
+        if t is not None:
+            _need(t, name, dt, dev)
+            if t.shape != (N,):
+                raise ValueError(f"{name} must be [N]")
+        ptrs.append(t.data_ptr() if t is not None else None)
+    if out is None:
+        out = torch.zeros((N, max(mb, 1)), dtype=torch.int64, device=dev)
+    else:
+        _need(out, "out", torch.int64, dev)
+        if out.dim() != 2 or out.shape[0] != N or out.shape[1] < mb:
+            raise ValueError(f"out must be [N, >= {mb}]")
     rc = library().pkv_prefix_block_hashes(
         tokens.data_ptr(), T, seq_lens.data_ptr(),
-        extra_keys.data_ptr() if extra_keys is not None else None, N, int(block_size),
-        out.data_ptr(), mb, _stream(dev, stream))
+        extra_keys.data_ptr() if extra_keys is not None else None, ptrs[0], ptrs[1], N,
+        int(block_size), out.data_ptr(), out.shape[1] if mb > 0 else 0, _stream(dev, stream))
     _check(rc, "prefix_block_hashes")
     return out[:, :mb]
 

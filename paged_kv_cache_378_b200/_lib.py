@@ -43,8 +43,8 @@ SIGNATURES = {
     "pkv_swap_blocks": (ctypes.c_int, [ctypes.POINTER(PkvCache), ctypes.POINTER(PkvCache),
                                        ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "pkv_prefix_block_hashes": (ctypes.c_int, [
-        ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
-        ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
+        ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "pkv_block_manager_step": (ctypes.c_int, [
         ctypes.POINTER(PkvBlockState), ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,

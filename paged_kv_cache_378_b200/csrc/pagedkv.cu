@@ -488,7 +488,8 @@ int pkv_swap_blocks(const pkv_cache_t* device_cache, const pkv_cache_t* host_cac
 }
 
 int pkv_prefix_block_hashes(const int32_t* tokens, int max_tokens, const int32_t* seq_lens,
-                            const uint64_t* extra_keys, int num_seqs, int block_size,
+                            const uint64_t* extra_keys, const int32_t* first_block,
+                            const uint64_t* parent_hashes, int num_seqs, int block_size,
                             uint64_t* hashes, int max_blocks, void* stream) {
     if (num_seqs < 0 || max_tokens < 0 || max_blocks < 0 || block_size <= 0) return PKV_ERR_SHAPE;
     if (num_seqs == 0 || max_blocks == 0) return PKV_OK;
@@ -499,7 +500,7 @@ int pkv_prefix_block_hashes(const int32_t* tokens, int max_tokens, const int32_t
     if (grid > cap) grid = cap;
     return launch_pdl(pkv::prefix_hash_kernel, dim3((unsigned)grid), dim3(per_cta * 32), 0,
                       (cudaStream_t)stream, tokens, (long long)max_tokens, seq_lens, extra_keys,
-                      num_seqs, block_size, hashes, max_blocks);
+                      first_block, parent_hashes, num_seqs, block_size, hashes, max_blocks);
 }
 
 int pkv_block_manager_step(const pkv_block_state_t* st, int num_seqs, int max_blocks_per_seq,

@@ -39,6 +39,8 @@ __device__ __forceinline__ uint64_t fnv_u64(uint64_t h, uint64_t v) {
 __global__ void __launch_bounds__(256)
 prefix_hash_kernel(const int32_t* __restrict__ tokens, long long row_stride,
                    const int32_t* __restrict__ seq_lens, const uint64_t* __restrict__ extra_keys,
+                   const int32_t* __restrict__ first_block,      // null: 0
+                   const uint64_t* __restrict__ parent_hashes,   // null: 0
                    int num_seqs, int block_size, uint64_t* __restrict__ hashes, int max_blocks) {
     pdl_launch_dependents();
     pdl_wait();
@@ -57,8 +59,12 @@ prefix_hash_kernel(const int32_t* __restrict__ tokens, long long row_stride,
         }
         const uint64_t key = extra_keys ? __ldg(extra_keys + s) : 0ull;
         const int32_t* row = tokens + (size_t)s * row_stride;
-        uint64_t parent = 0;
-        for (long long b0 = 0; b0 < full; b0 += 32) {
+        // resume: blocks before `start` are hashed already; parent is the hash
+        // of block start - 1 (ignored at start 0)
+        long long start = first_block ? __ldg(first_block + s) : 0;
+        if (start < 0) start = 0;
+        uint64_t parent = (start > 0 && parent_hashes) ? __ldg(parent_hashes + s) : 0ull;
+        for (long long b0 = start; b0 < full; b0 += 32) {
             const long long b = b0 + lane;
             uint64_t c = 0;
             if (b < full) {

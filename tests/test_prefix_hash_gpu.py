@@ -77,3 +77,30 @@ def test_full_step_sampled():
     tokens = token_ids(w)
     rng = np.random.default_rng(5)
     _check(tokens, w.seq_lens, w.block_size, None, rng.choice(w.num_seqs, 12, replace=False))
+
+
+def test_resume_from_a_parent_hash():
+    # hashing from block k with the stored hash of block k-1 gives the same
+    # hashes as hashing the whole prefix; blocks before k are left untouched
+    # (the decode case: only the block that just became full)
+    rng = np.random.default_rng(9)
+    N, B, T = 50, 16, 640
+    tokens = rng.integers(0, 128256, (N, T)).astype(np.int32)
+    lens = rng.integers(0, T + 1, N).astype(np.int32)
+    tok_d, len_d = torch.from_numpy(tokens).cuda(), torch.from_numpy(lens).cuda()
+    whole = pkv.prefix_block_hashes(tok_d, len_d, B).cpu().numpy()
+    nfull = lens // B
+    first = np.array([rng.integers(0, n + 1) for n in nfull], np.int32)
+    first[:4] = [0, nfull[1], max(nfull[2] - 1, 0), nfull[3]]
+    parents = np.array([whole[s, first[s] - 1] if first[s] > 0 else 0 for s in range(N)], np.int64)
+    out = torch.full((N, T // B), 7, dtype=torch.int64, device="cuda")
+    res = pkv.prefix_block_hashes(tok_d, len_d, B, first_block=torch.from_numpy(first).cuda(),
+                                  parent_hashes=torch.from_numpy(parents).cuda(), out=out)
+    torch.cuda.synchronize()
+    assert pkv.get_device_status(reset=True) == 0
+    res = res.cpu().numpy()
+    for s in range(N):
+        assert np.array_equal(res[s, first[s]:nfull[s]], whole[s, first[s]:nfull[s]]), s
+        assert np.all(res[s, :first[s]] == 7) and np.all(res[s, nfull[s]:] == 7), s
+        want = ph.prefix_block_hashes(tokens[s].tolist(), int(lens[s]), B)
+        assert [_u64(x) for x in res[s, first[s]:nfull[s]]] == want[first[s]:], s
