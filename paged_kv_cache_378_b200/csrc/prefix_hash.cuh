@@ -23,7 +23,17 @@ namespace pkv {
 constexpr uint64_t FNV64_OFFSET = 0xCBF29CE484222325ull;
 constexpr uint64_t FNV64_PRIME = 0x100000001B3ull;
 
-__device__ __forceinline__ uint64_t fnv_byte(uint64_t h, uint32_t b) { return (h ^ b) * FNV64_PRIME; }
+// One FNV-1a step, (h ^ b) * FNV64_PRIME mod 2^64, on 32-bit halves: the
+// prime is 2^40 + 0x1b3, so with x = h ^ b = (hi, lo)
+//   x * prime = lo * 0x1b3 + ((hi * 0x1b3 + (lo << 8)) mod 2^32) * 2^32,
+// one wide multiply and one short one instead of a general 64-bit product.
+__device__ __forceinline__ uint64_t fnv_byte(uint64_t h, uint32_t b) {
+    const uint32_t lo = (uint32_t)h ^ b;
+    const uint32_t hi = (uint32_t)(h >> 32);
+    const uint64_t t = (uint64_t)lo * 0x1b3u;
+    const uint32_t nhi = (uint32_t)(t >> 32) + hi * 0x1b3u + (lo << 8);
+    return ((uint64_t)nhi << 32) | (uint32_t)t;
+}
 
 __device__ __forceinline__ uint64_t fnv_u32(uint64_t h, uint32_t v) {
 #pragma unroll
