@@ -42,6 +42,7 @@ METRIC = "paged decode attention KV GB/s and % of HBM peak; decode tokens/s per 
 UNIT = "GB/s"
 DEFAULT_WORKLOAD = "continuous_batch"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0   # the ~8 TB/s the 70 % bandwidth target is stated against
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "attention_traffic.json")
 EVENT_EVERY = 8            # attention events on every 8th timed step
 # device sources of the attention kernel: a committed DRAM-traffic capture
@@ -352,15 +353,36 @@ STEP_TEXT = {"cow": "per layer one launch: copy-on-write of shared tails, append
              "two-call": "block_copy, then per layer kv_append and attention launches"}
 
 
-def workload_config(pkv, key, spec, w, B, part, world, mode):
+L2_TEXT = ("inputs larger than L2: each step reads its own copy of the KV pools, rotating "
+           "through copies that total at least 4x the L2 size")
+
+
+def attention_tile_tokens(head_dim, block_size):
+    """Tokens per pipeline stage of the attention kernel: a whole block at 32,
+    32 at head_dim 64 with blocks of 8 or more, else 16."""
+    if block_size >= 32:
+        return block_size
+    return 32 if head_dim == 64 and block_size >= 8 else 16
+
+
+def rounded_partition(spec, B, requested):
+    """The longest work range the attention call uses for ``requested``
+    tokens (0 = no cap): rounded up to the kernel's tile.  Plain host
+    arithmetic, so the reference arm can print it without the library."""
+    if requested <= 0:
+        return 0
+    t = attention_tile_tokens(spec.head_dim, B)
+    return -(-int(requested) // t) * t
+
+
+def workload_config(key, spec, w, B, part, world, mode):
     """The ``config`` object both arms print for a workload."""
     return {"workload": key, "title": spec.title, "num_seqs": w.num_seqs,
             "num_layers": spec.num_layers, "q_heads": spec.num_q_heads,
             "kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim, "block_size": B,
-            "partition_tokens": pkv.partition_tokens(w.num_seqs, spec.num_kv_heads,
-                                                     spec.head_dim, w.max_blocks, B, part),
+            "partition_tokens": rounded_partition(spec, B, part),
             "parallelism": f"dp{world} (independent batches, no collective)",
-            "step": STEP_TEXT[mode]}
+            "step": STEP_TEXT[mode], "l2": L2_TEXT}
 
 
 def cow_sources(w):
@@ -476,6 +498,48 @@ def prefix_hash_timing(pkv, w, device, iters=50):
             "token_bytes_gbs": blocks * w.block_size * 4 / (us * 1e-6) / 1e9,
             "what": "FNV-1a 64 chain hash of every full block (parent hash, block tokens, "
                     "extra key), one warp per sequence"}
+
+
+def prefix_hash_decode_timing(pkv, w, device, iters=50):
+    """Mean device time of the per-step (decode) form of the prefix hash: each
+    sequence hashes only its newest full block, resuming the chain from the
+    stored hash of the block before it (``first_block``/``parent_hashes``).
+    Every sequence is given one block to hash (the last full one), the most a
+    decode step can ask for."""
+    from workload import token_ids
+    tok = torch.from_numpy(token_ids(w)).to(device)
+    lens_np = w.seq_lens.astype(np.int64)
+    full = lens_np // w.block_size
+    first = np.maximum(full - 1, 0).astype(np.int32)
+    lens = torch.from_numpy(w.seq_lens).to(device)
+    first_d = torch.from_numpy(first).to(device)
+    N, T = tok.shape
+    mb = T // w.block_size
+    parents = torch.zeros(N, dtype=torch.int64, device=device)   # stored hashes (values do not matter for time)
+    out = torch.zeros((N, mb), dtype=torch.int64, device=device)
+    busy = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    lib = pkv.library()
+    stream = torch.cuda.current_stream(device)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(iters)]
+    for i in range(iters + 3):
+        busy.zero_()
+        if i >= 3:
+            evs[i - 3][0].record(stream)
+        if lib.pkv_prefix_block_hashes(tok.data_ptr(), T, lens.data_ptr(), None, first_d.data_ptr(),
+                                       parents.data_ptr(), N, w.block_size, out.data_ptr(), mb, sp):
+            raise SystemExit("prefix hash (decode form) refused its arguments")
+        if i >= 3:
+            evs[i - 3][1].record(stream)
+    torch.cuda.synchronize(device)
+    if pkv.get_device_status(reset=True):
+        raise SystemExit("device status raised by the prefix hash (decode form)")
+    us = sum(a.elapsed_time(b) for a, b in evs) / iters * 1e3
+    blocks = int((full > 0).sum())
+    return {"us": us, "blocks": blocks, "blocks_per_s": blocks / (us * 1e-6),
+            "what": "decode form: one newly full block per sequence, chain resumed from the "
+                    "stored parent hash"}
 
 
 def swap_timing(pkv, w, device, blocks=1024, iters=10):
@@ -626,6 +690,17 @@ def limit_blas_threads():
         return None
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def host_workload(key, block_size, seed):
     w = make_workload(key, block_size=block_size, seed=seed, device="cpu", poison=False)
     host = dict(k=_u16(w.k_pool), v=_u16(w.v_pool), q=_u16(w.q), k_new=_u16(w.k_new),
@@ -633,10 +708,11 @@ def host_workload(key, block_size, seed):
     return w, host
 
 
-def cpu_baseline(key, block_size, seed, unique_bytes, min_seconds=10.0):
+def cpu_baseline_single(w, host, unique_bytes, min_seconds=10.0):
+    """The oracle's whole step, one thread (BLAS pinned to 1), repeated for
+    about ``min_seconds``."""
     from oracle import attention as oa
     lim = limit_blas_threads()
-    w, host = host_workload(key, block_size, seed)
     n = 0
     t0 = time.perf_counter()
     while True:
@@ -653,8 +729,121 @@ def cpu_baseline(key, block_size, seed, unique_bytes, min_seconds=10.0):
                       f"{dt:.2f} s per step, numpy fp64, 1 thread"}
 
 
+# -- the oracle over every host core: a process pool over sequences --------------
+# Workers are started with ``spawn`` (never forked from a process that has
+# touched the GPU) and read the step's pools from shared memory.
+
+_POOL_STATE = {}
+
+
+def _pool_worker_init(shm_specs, meta):
+    from multiprocessing import shared_memory
+    limit_blas_threads()
+    arrays, handles = {}, []
+    for k, (name, shape, dtype) in shm_specs.items():
+        shm = shared_memory.SharedMemory(name=name)
+        handles.append(shm)
+        arrays[k] = np.ndarray(shape, dtype=np.dtype(dtype), buffer=shm.buf)
+    _POOL_STATE.update(arrays)
+    _POOL_STATE["_handles"] = handles
+    _POOL_STATE["meta"] = meta
+
+
+def _pool_worker_attention(idx):
+    """The oracle's attention for sequences ``idx``, every layer."""
+    from oracle import attention as oa
+    P = _POOL_STATE
+    m = P["meta"]
+    idx = np.asarray(idx, dtype=np.int64)
+    for layer in range(m["L"]):
+        oa.paged_decode_attention(P["q"][layer][idx], P["k2"][layer], P["v2"][layer],
+                                  P["tables"][idx], P["lens"][idx], m["B"], m["scale"])
+    return len(idx)
+
+
+def cpu_baseline_all_cores(w, host, unique_bytes, min_seconds=10.0):
+    """The oracle's whole step with its attention spread over a ``spawn``
+    process pool, one worker per core of ``os.sched_getaffinity(0)``: the
+    parent runs the oracle's block_copy and kv_append, the workers the
+    oracle's attention on balanced groups of sequences.  Returns None where
+    a pool cannot be started."""
+    import multiprocessing as mp
+    from multiprocessing import shared_memory
+    from oracle import attention as oa
+    cores = len(os.sched_getaffinity(0))
+    L = w.spec.num_layers
+    kp, vp = oa.block_copy(host["k"], host["v"], w.copy_pairs)
+    k2 = np.empty_like(kp)
+    v2 = np.empty_like(vp)
+    for layer in range(L):
+        k2[layer], v2[layer] = oa.kv_append(kp[layer], vp[layer], host["k_new"][layer],
+                                            host["v_new"][layer], w.slot_mapping, w.block_size)
+    arrays = {"q": host["q"], "k2": k2, "v2": v2, "tables": w.block_tables, "lens": w.seq_lens}
+    shms, specs = [], {}
+    try:
+        for k, a in arrays.items():
+            shm = shared_memory.SharedMemory(create=True, size=max(1, a.nbytes))
+            shms.append(shm)
+            np.ndarray(a.shape, dtype=a.dtype, buffer=shm.buf)[...] = a
+            specs[k] = (shm.name, a.shape, a.dtype.str)
+        # groups of sequences of about equal KV bytes, 4 per worker
+        lens = w.seq_lens.astype(np.int64)
+        ngroups = max(1, min(w.num_seqs, 4 * cores))
+        groups = [[] for _ in range(ngroups)]
+        load = np.zeros(ngroups)
+        for s in np.argsort(-lens, kind="stable").tolist():
+            g = int(np.argmin(load))
+            groups[g].append(s)
+            load[g] += lens[s] + 1
+        groups = [g for g in groups if g]
+        meta = {"L": L, "B": w.block_size, "scale": w.spec.scale}
+        ctx = mp.get_context("spawn")
+        with ctx.Pool(cores, initializer=_pool_worker_init, initargs=(specs, meta)) as pool:
+            pool.map(_pool_worker_attention, [[0]] * cores)          # start and warm every worker
+            lim = limit_blas_threads()
+            n = 0
+            t0 = time.perf_counter()
+            while True:
+                kq, vq = oa.block_copy(host["k"], host["v"], w.copy_pairs)
+                for layer in range(L):
+                    oa.kv_append(kq[layer], vq[layer], host["k_new"][layer], host["v_new"][layer],
+                                 w.slot_mapping, w.block_size)
+                pool.map(_pool_worker_attention, groups, chunksize=1)
+                n += 1
+                if time.perf_counter() - t0 >= min_seconds:
+                    break
+            dt = (time.perf_counter() - t0) / n
+            del lim
+    except (OSError, RuntimeError) as e:
+        return {"unavailable": f"{type(e).__name__}: {e}"}
+    finally:
+        for shm in shms:
+            shm.close()
+            shm.unlink()
+    return {"value": unique_bytes * L / dt / 1e9, "unit": UNIT, "cores": cores,
+            "kind": "oracle", "cpu_model": cpu_model(),
+            "sample": f"the whole step of this workload (all {w.num_seqs} sequences, "
+                      f"{L} layer(s)): block_copy and kv_append in the parent, attention over "
+                      f"{len(groups)} balanced groups of sequences on a spawn pool of {cores} "
+                      f"worker processes (one per core of sched_getaffinity, BLAS 1 thread each); "
+                      f"repeated {n}x, {dt:.2f} s per step, numpy fp64"}
+
+
+def cpu_baseline(key, block_size, seed, unique_bytes, min_seconds=10.0):
+    """Both oracle timings on the host: one thread, and every core."""
+    w, host = host_workload(key, block_size, seed)
+    one = cpu_baseline_single(w, host, unique_bytes, min_seconds)
+    every = cpu_baseline_all_cores(w, host, unique_bytes, min_seconds)
+    if every is None or "unavailable" in every:
+        one["all_cores"] = every
+        return one
+    every["single_thread"] = one
+    return every
+
+
 def run_reference(args):
-    """--impl reference: the oracle timed as it stands on the host cores."""
+    """--impl reference: the oracle timed as it stands on the host cores.
+    Touches neither the GPU nor this repository's library."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
@@ -663,11 +852,8 @@ def run_reference(args):
     B = args.block_size or spec.block_size
     lim = limit_blas_threads()
     w, host = host_workload(args.workload, B, spec.seed)
-    # the same config object our arm prints (the library's partition rounding
-    # is host arithmetic; nothing runs on the GPU here)
-    import paged_kv_cache_378_b200 as pkv
     part = spec.partition_tokens if args.partition < 0 else args.partition
-    ref_config = workload_config(pkv, args.workload, spec, w, B, part,
+    ref_config = workload_config(args.workload, spec, w, B, part,
                                  int(os.environ.get("WORLD_SIZE", "1")), args.step)
     kp, vp = oa.block_copy(host["k"], host["v"], w.copy_pairs)
     k2, v2 = oa.kv_append(kp[0], vp[0], host["k_new"][0], host["v_new"][0], w.slot_mapping,
@@ -713,6 +899,117 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# measurement of a step made of attention launches only (copy-on-write folded in)
+# ---------------------------------------------------------------------------
+
+def algorithmic_bytes(w, spec, B, gs, unique_bytes):
+    """Algorithmic bytes of one attention launch (one layer): unique K/V, q
+    and out, tables and lengths, and with the fused append the new tokens'
+    K/V read and stored, and with the folded copy-on-write the copied tail
+    blocks written."""
+    q_out = 2 * w.num_seqs * spec.num_q_heads * spec.head_dim * 2
+    meta = w.block_tables.nbytes + w.seq_lens.nbytes
+    append = 2 * (2 * w.num_seqs * spec.num_kv_heads * spec.head_dim * 2) if gs.fused else 0
+    cow = (gs.npairs * spec.num_kv_heads * B * spec.head_dim * 2 * 2) if gs.mode == "cow" else 0
+    return {"unique_kv": unique_bytes, "q_out": q_out, "tables_lengths": meta,
+            "append": append, "copy_on_write": cow,
+            "total": unique_bytes + q_out + meta + append + cow}
+
+
+def region_ms(gs, steps, first=0):
+    """Device time of ``steps`` chained steps (CUDA events on the launching stream)."""
+    fast = gs.prepared()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(gs.stream)
+    for i in range(steps):
+        fast(first + i)
+    e1.record(gs.stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def launch_stats(gs, steps, first=0):
+    """Per-launch attention times from a separate, untimed pass with events
+    around every launch (each launch then runs alone: no overlap with the
+    one before it), in microseconds."""
+    L = gs.L
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(L)] for _ in range(steps)]
+    for i in range(steps):
+        gs.run(first + i, evs[i])
+    torch.cuda.synchronize(gs.device)
+    us = sorted(a.elapsed_time(b) * 1e3 for row in evs for a, b in row)
+
+    def q(p):
+        return us[min(len(us) - 1, int(round(p * (len(us) - 1))))]
+    return {"launches": len(us), "median_us": q(0.5), "p10_us": q(0.1), "p90_us": q(0.9),
+            "min_us": us[0], "max_us": us[-1],
+            "what": "each attention launch bracketed by CUDA events in a separate pass "
+                    "(launches then do not overlap their neighbours)"}
+
+
+def peak_fractions(gbs, peak):
+    return {"pct_of_8tbs": 100.0 * gbs / NOMINAL_HBM_GBS, "pct_of_measured": 100.0 * gbs / peak}
+
+
+def measure_config(pkv, key, B, part, device, sampler, peak, peak_kind, min_region_s=0.3):
+    """One workload at one block size through the default step (one launch per
+    layer: copy-on-write, append, attention): value, roofline, clocks and
+    per-launch statistics, for the ``per_config`` part of the line."""
+    spec = get_spec(key)
+    w = make_workload(key, block_size=B, seed=spec.seed, device=device, poison=False)
+    unique = w.unique_kv_bytes_read()
+    pool_bytes = 2 * w.k_pool.numel() * w.k_pool.element_size()
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    nrep = max(1, min(16, math.ceil(4 * l2 / pool_bytes)))
+    replicas = [(w.k_pool, w.v_pool)] + [(w.k_pool.clone(), w.v_pool.clone())
+                                         for _ in range(nrep - 1)]
+    gs = GpuStep(pkv, w, replicas, part, device, mode="cow")
+    pkv.get_device_status(reset=True)
+    for i in range(5):
+        gs.run(i)
+    est = region_ms(gs, 3, 5) / 3
+    steps = max(20, int(math.ceil(min_region_s * 1e3 / max(est, 1e-3))))
+    torch.cuda.synchronize(device)
+    wall0 = time.time()
+    ms = region_ms(gs, steps, 8)
+    wall1 = time.time()
+    stats = launch_stats(gs, max(8, min(200, int(math.ceil(200 / spec.num_layers)))), 8 + steps)
+    status = pkv.get_device_status(reset=True)
+    if status:
+        raise SystemExit(f"device status {status:#x} raised while measuring {key} B={B}")
+    ms_step = ms / steps
+    value = unique * spec.num_layers / (ms_step * 1e-3) / 1e9
+    alg = algorithmic_bytes(w, spec, B, gs, unique)
+    launch_us = ms_step * 1e3 / spec.num_layers
+    achieved = alg["total"] / (launch_us * 1e-6) / 1e9
+    out = {"workload": key, "block_size": B,
+           "partition_tokens": rounded_partition(spec, B, part),
+           "num_seqs": w.num_seqs, "num_layers": spec.num_layers,
+           "value": value, "unit": UNIT, "steps": steps, "ms_per_step": ms_step,
+           "decode_tokens_per_s_per_layer": w.num_seqs * spec.num_layers / (ms_step * 1e-3),
+           "kv_bytes_per_step": {"unique": unique * spec.num_layers,
+                                 "logical": w.kv_bytes_read() * spec.num_layers},
+           **peak_fractions(value, peak),
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                        "frac": achieved / peak, "kernel": "paged_attention_kernel",
+                        "alg_bytes_per_launch": alg, "avg_launch_us": launch_us,
+                        "peak_source": f"{peak_kind} hbm_gbs"},
+           "launch_stats": stats,
+           "clocks": sampler.summary(wall0 - 0.05, wall1 + 0.05),
+           "l2": f"{nrep} rotating copies of the KV pools, {nrep * pool_bytes / 1e9:.2f} GB vs "
+                 f"{l2 / 1e6:.0f} MB L2"}
+    del gs, replicas, w
+    torch.cuda.empty_cache()
+    return out
+
+
+PER_CONFIG = [("llama1b_layer", 16, -1), ("long_context", 16, -1), ("long_context", 16, 0),
+              ("full_step", 8, -1), ("full_step", 16, -1), ("full_step", 32, -1)]
+
+
+# ---------------------------------------------------------------------------
 # main (our arm)
 # ---------------------------------------------------------------------------
 
@@ -727,6 +1024,10 @@ def main():
     ap.add_argument("--partition", type=int, default=-1, help="-1: the workload's, 0: library default")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the other workloads' lines (per_config)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the block-manager, swap and prefix-hash timings")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--soak-seconds", type=float, default=1.5)
     ap.add_argument("--step", choices=["cow", "fused", "two-call"], default="cow",
@@ -742,6 +1043,20 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    spec = get_spec(args.workload)
+    B = args.block_size or spec.block_size
+    part = spec.partition_tokens if args.partition < 0 else args.partition
+    seed = rank_seed(spec.seed, rank)
+
+    # cpu baseline first, before this process touches the GPU (its pool is
+    # spawned; rank 0 at N = 1 only)
+    w_meta = make_workload(args.workload, block_size=B, seed=seed, values=False)
+    unique_bytes = w_meta.unique_kv_bytes_read()
+    logical_bytes = w_meta.kv_bytes_read()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, B, seed, unique_bytes)
+
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
     torch.cuda.set_device(local)
@@ -755,22 +1070,13 @@ def main():
 
     import paged_kv_cache_378_b200 as pkv
 
-    spec = get_spec(args.workload)
-    B = args.block_size or spec.block_size
-    part = spec.partition_tokens if args.partition < 0 else args.partition
-    seed = rank_seed(spec.seed, rank)
-
-    sampler = ClockSampler(pci_bus_id(local)).start()   # warms up while the inputs are built
-
-    # cpu baseline first, before the GPU is busy (rank 0 at N = 1 only)
-    w_meta = make_workload(args.workload, block_size=B, seed=seed, values=False)
-    unique_bytes = w_meta.unique_kv_bytes_read()
-    logical_bytes = w_meta.kv_bytes_read()
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(args.workload, B, seed, unique_bytes)
+    sampler = ClockSampler(pci_bus_id(local)).start()
 
     w = make_workload(args.workload, block_size=B, seed=seed, device=device, poison=False)
+    rounded = pkv.partition_tokens(w.num_seqs, spec.num_kv_heads, spec.head_dim, w.max_blocks, B,
+                                   part)
+    if rounded != rounded_partition(spec, B, part):
+        raise SystemExit("partition rounding differs from the library's")
     pool_bytes = 2 * w.k_pool.numel() * w.k_pool.element_size()
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     nrep = max(1, min(16, math.ceil(4 * l2 / pool_bytes)))
@@ -825,7 +1131,6 @@ def main():
                 i += 1
             torch.cuda.synchronize(device)
         soak_until = time.time()
-    sampler.stop()
     clocks = sampler.summary(wall0 - 0.05, soak_until + 0.05)
     clocks["window"] = "timed region" if soak_until == wall1 else "timed region + untimed soak"
     status = pkv.get_device_status(reset=True)
@@ -839,6 +1144,8 @@ def main():
         attn_ms = [a.elapsed_time(b) for a, b in evs]
         sampling = f"attention bracketed on every {EVENT_EVERY}th timed step"
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
+    # per-launch distribution from a separate untimed pass (every launch alone)
+    stats = launch_stats(gs, max(50, min(500, args.steps)), args.steps + 10**6)
 
     # totals over ranks: device time is the max, work is the sum
     ms_max, bytes_total, seqs_total = combine_over_ranks(
@@ -856,49 +1163,62 @@ def main():
                "pipeline": "three buffer sets: uploads and downloads of neighbouring steps on copy streams while step i computes",
                "host_cpus": f"{ncpu} GPU-local CPUs" if ncpu else "affinity unchanged"}
 
-    bm_us = block_manager_timing(pkv, w, device) if w.num_seqs <= 4096 else None
-    swap = swap_timing(pkv, w, device)
-    phash = prefix_hash_timing(pkv, w, device)
+    extras = {}
+    if not args.no_extras:
+        bm_us = block_manager_timing(pkv, w, device) if w.num_seqs <= 4096 else None
+        extras["swap"] = swap_timing(pkv, w, device)
+        extras["prefix_hash"] = prefix_hash_timing(pkv, w, device)
+        extras["prefix_hash_decode"] = prefix_hash_decode_timing(pkv, w, device)
+        extras["block_manager"] = None if bm_us is None else {
+            "us_per_step": bm_us, "num_seqs": w.num_seqs,
+            "what": "device block-manager step (slot mapping, copy-on-write decisions, block "
+                    "allocation) timed alone on this step's pre-step state, restored between launches"}
 
     peak, peak_kind = load_peak()
-    q_out_bytes = 2 * w.num_seqs * spec.num_q_heads * spec.head_dim * 2
-    meta_bytes = w.block_tables.nbytes + w.seq_lens.nbytes
-    # the fused kernel also reads k_new/v_new and stores them in their slots
-    append_bytes = 2 * (2 * w.num_seqs * spec.num_kv_heads * spec.head_dim * 2) if gs.fused else 0
-    # with the copy-on-write folded in, the kernel also writes each copied tail
-    # block (this layer, K and V); its source is read as the tail itself
-    cow_bytes = (gs.npairs * spec.num_kv_heads * B * spec.head_dim * 2 * 2
-                 if gs.mode == "cow" else 0)
-    alg_bytes = unique_bytes + q_out_bytes + meta_bytes + append_bytes + cow_bytes
-    achieved = alg_bytes / (attn_avg_ms * 1e-3) / 1e9
+    alg = algorithmic_bytes(w, spec, B, gs, unique_bytes)
+    achieved = alg["total"] / (attn_avg_ms * 1e-3) / 1e9
     traffic = load_traffic(args.workload, B, gs.mode)
+    launches_per_step = gs.launches_per_step
+    del gs, replicas, w
+    torch.cuda.empty_cache()
+
+    # the other workloads, each through the same step (rank 0 at N = 1 only;
+    # ranks of a multi-GPU run take the same collective steps without these)
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        per_config = []
+        for key, bs, p in PER_CONFIG:
+            sp = get_spec(key)
+            per_config.append(measure_config(pkv, key, bs, sp.partition_tokens if p < 0 else p,
+                                             device, sampler, peak, peak_kind))
+    sampler.stop()
+
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(pkv, args.workload, spec, w, B, part, world, gs.mode),
-                       l2=f"inputs larger than L2: {nrep} rotating copies of the KV pools, "
-                          f"{nrep * pool_bytes / 1e9:.2f} GB vs {l2 / 1e6:.0f} MB L2"),
+        "config": workload_config(args.workload, spec, w_meta, B, part, world, args.step),
+        "l2_detail": f"{nrep} rotating copies of the KV pools, {nrep * pool_bytes / 1e9:.2f} GB vs "
+                     f"{l2 / 1e6:.0f} MB L2",
         "pct_hbm_peak": 100.0 * value / peak,
+        **peak_fractions(value, peak),
         # one token per sequence per layer: N x L tokens cross a layer per step
         "decode_tokens_per_s_per_layer": seqs_total * spec.num_layers / (ms_per_step * 1e-3),
         "kv_bytes_per_step": {"unique": unique_bytes * spec.num_layers,
                               "logical": logical_bytes * spec.num_layers},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "paged_attention_kernel", "alg_bytes_per_launch": alg_bytes,
+                     "kernel": "paged_attention_kernel", "alg_bytes_per_launch": alg["total"],
+                     "alg_bytes_parts": alg,
                      "avg_launch_us": attn_avg_ms * 1e3, "peak_source": f"{peak_kind} hbm_gbs",
                      "timed_launches": len(attn_ms),
                      "event_sampling": sampling},
+        "launch_stats": stats,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "swap": swap,
-        "prefix_hash": phash,
-        "block_manager": None if bm_us is None else {
-            "us_per_step": bm_us, "num_seqs": w.num_seqs,
-            "what": "device block-manager step (slot mapping, copy-on-write decisions, block "
-                    "allocation) timed alone on this step's pre-step state, restored between launches"},
-        "gpu_launches": gs.launches_per_step * args.steps,
+        **extras,
+        "per_config": per_config,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
     if rank == 0:

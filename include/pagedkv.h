@@ -80,6 +80,10 @@ extern "C" {
 /* size of the device buffer behind pkv_paged_decode_attention_noalloc */
 #define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
 
+/* cow_src value: this sequence appends nothing in this step (written by an
+ * aborted pkv_block_manager_step; see pkv_append_paged_decode_attention) */
+#define PKV_COW_NO_APPEND (-2)
+
 /* device-side status bits (pkv_get_device_status) */
 #define PKV_DEV_RANGE    0x1u  /* block id or slot outside the pool: access skipped */
 #define PKV_DEV_LENGTH   0x2u  /* seq_len above max_blocks_per_seq * block_size: clamped */
@@ -191,8 +195,12 @@ int pkv_swap_blocks(const pkv_cache_t* device_cache, const pkv_cache_t* host_cac
  *   first_block  device int32 [num_seqs], or NULL for 0: hash only blocks
  *                first_block[s] .. seq_lens/B - 1 (resuming, e.g. in decode
  *                only the block that just became full)
- *   parent_hashes device uint64 [num_seqs], or NULL: hash of block
- *                first_block[s] - 1 (unused where first_block[s] is 0)
+ *   parent_hashes device uint64 [num_seqs]: hash of block first_block[s] - 1
+ *                (unused where first_block[s] is 0).  Required whenever
+ *                first_block is given (PKV_ERR_NULL otherwise: a chain
+ *                restarted from 0 would give block k the hash of a first
+ *                block with the same tokens, a false prefix match); may be
+ *                NULL when first_block is NULL.
  *   hashes       device uint64 [num_seqs][max_blocks] out; entries outside
  *                [first_block, full blocks) are not written
  * A length above max_tokens, or more full blocks than max_blocks, sets
@@ -240,10 +248,16 @@ typedef struct pkv_block_state {
  *                  form pkv_append_paged_decode_attention takes
  * On return the tables, lengths (+1), counts and free state are updated.
  * num_seqs <= 4096 (PKV_ERR_UNSUPPORTED above).  If the free blocks do not
- * suffice, or an order entry, a length or a tail block id is out of range,
- * the kernel sets PKV_DEV_NOBLOCKS / PKV_DEV_RANGE / PKV_DEV_LENGTH and
- * changes nothing.  The kernel does not release its dependents early, so an
- * attention launch that follows on the stream reads the new lengths.
+ * suffice, or an order entry, a length, a tail block id or a free-ring entry
+ * is out of range, the kernel sets PKV_DEV_NOBLOCKS / PKV_DEV_RANGE /
+ * PKV_DEV_LENGTH and changes no state (tables, lengths, counts, free state).
+ * It still writes its outputs, so that work already queued behind it on the
+ * stream does no harm before the host sees the status: every slot_mapping
+ * entry -1 (pkv_kv_append skips it), *num_pairs = 0 (no copy), and, when
+ * cow_src is given, cow_src[s] = PKV_COW_NO_APPEND for every sequence (the
+ * fused pkv_append_paged_decode_attention then appends and copies nothing).
+ * The kernel does not release its dependents early, so an attention launch
+ * that follows on the stream reads the new lengths.
  */
 int pkv_block_manager_step(const pkv_block_state_t* state, int num_seqs,
                            int max_blocks_per_seq, int num_blocks, int block_size,
@@ -348,7 +362,12 @@ int pkv_paged_decode_attention(const pkv_cache_t* cache, int layer,
  *                  block, this layer, every kv head, K and V, to the tail
  *                  block with the new token in place -- what pkv_block_copy
  *                  of (cow_src[s], tail) for this layer followed by
- *                  pkv_kv_append would leave.  -1: no copy.  Read, like
+ *                  pkv_kv_append would leave.  -1: no copy.
+ *                  PKV_COW_NO_APPEND (-2): sequence s appends nothing and
+ *                  copies nothing in this launch (its attention reads the
+ *                  pool as it is); an aborted pkv_block_manager_step writes
+ *                  this for every sequence, so a device-only step chained
+ *                  behind it leaves the pools untouched.  Read, like
  *                  seq_lens and the tables, before the wait on the previous
  *                  kernel.
  *   other arguments as pkv_paged_decode_attention.
@@ -408,6 +427,19 @@ int pkv_paged_decode_attention_noalloc(const pkv_cache_t* cache, int layer,
                                        int partition_tokens, void* stream);
 
 /*
+ * pkv_set_wait_limit_ns -- how long the attention kernel's bounded wait for a
+ * staged tile may last on the current device before it gives up with
+ * PKV_DEV_TIMEOUT (0 = the default, 2 seconds).  A timed-out warp still
+ * waits (up to half a second, a fixed limit) for the copies it has in
+ * flight before it exits, so no copy outlives the launch.  A short limit
+ * turns a stuck launch into an error status sooner; tests use a limit of a
+ * few nanoseconds to drive the timeout path without any fault.  Synchronous
+ * (a copy to a device variable); affects launches made after it returns.
+ * After a timeout, zero the workspace again (pkv_workspace_init).
+ */
+int pkv_set_wait_limit_ns(unsigned long long limit_ns);
+
+/*
  * pkv_get_device_status -- read (and with reset != 0, clear) the device status
  * word of the current device.  Synchronises the device first.
  */
@@ -418,6 +450,11 @@ const char* pkv_strerror(int code);
 
 /* pkv_abi_version -- PKV_ABI_VERSION of the loaded library. */
 int pkv_abi_version(void);
+
+/* pkv_build_hash -- 16 hex digits identifying the sources, header and
+ * compiler flags this library was built from (static string).  The Python
+ * loader rebuilds the library when it differs from the checkout's. */
+const char* pkv_build_hash(void);
 
 #ifdef __cplusplus
 }

@@ -31,13 +31,15 @@ __all__ = [
     "append_paged_decode_attention", "BlockState", "block_manager_step", "swap_blocks",
     "SWAP_OUT", "SWAP_IN", "prefix_block_hashes",
     "attention_workspace_bytes", "partition_tokens", "make_workspace",
-    "get_device_status", "library", "DEV_RANGE", "DEV_LENGTH", "DEV_TIMEOUT", "DEV_NOBLOCKS",
+    "get_device_status", "set_wait_limit_ns", "workspace_init", "library", "DEV_RANGE",
+    "DEV_LENGTH", "DEV_TIMEOUT", "DEV_NOBLOCKS", "COW_NO_APPEND",
 ]
 
 DEV_RANGE = 0x1
 DEV_LENGTH = 0x2
 DEV_TIMEOUT = 0x4
 DEV_NOBLOCKS = 0x8
+COW_NO_APPEND = -2      # cow_src entry: the sequence appends nothing this step
 
 
 class PagedKVError(RuntimeError):
@@ -168,16 +170,19 @@ def prefix_block_hashes(tokens, seq_lens, block_size, extra_keys=None, max_block
             if t.shape != (N,):
                 raise ValueError(f"{name} must be [N]")
         ptrs.append(t.data_ptr() if t is not None else None)
+    if first_block is not None and parent_hashes is None:
+        raise ValueError("first_block needs parent_hashes (the stored hash of the block "
+                         "before each sequence's first one)")
     if out is None:
         out = torch.zeros((N, max(mb, 1)), dtype=torch.int64, device=dev)
     else:
         _need(out, "out", torch.int64, dev)
-        if out.dim() != 2 or out.shape[0] != N or out.shape[1] < mb:
-            raise ValueError(f"out must be [N, >= {mb}]")
+        if out.dim() != 2 or out.shape[0] != N or out.shape[1] != max(mb, 1):
+            raise ValueError(f"out must be [N, {max(mb, 1)}] (max_blocks columns)")
     rc = library().pkv_prefix_block_hashes(
         tokens.data_ptr(), T, seq_lens.data_ptr(),
         extra_keys.data_ptr() if extra_keys is not None else None, ptrs[0], ptrs[1], N,
-        int(block_size), out.data_ptr(), out.shape[1] if mb > 0 else 0, _stream(dev, stream))
+        int(block_size), out.data_ptr(), mb, _stream(dev, stream))
     _check(rc, "prefix_block_hashes")
     return out[:, :mb]
 
@@ -366,6 +371,20 @@ def append_paged_decode_attention(k_new, v_new, q, k_pool, v_pool, block_tables,
         ws_bytes, int(partition_tokens), _stream(dev, stream))
     _check(rc, "append_paged_decode_attention")
     return out
+
+
+def set_wait_limit_ns(limit_ns=0):
+    """Limit (ns) of the attention kernel's bounded wait for a staged tile on
+    the current device; 0 restores the default (2 s).  A launch whose wait
+    runs out sets DEV_TIMEOUT; zero its workspace again afterwards."""
+    _check(library().pkv_set_wait_limit_ns(int(limit_ns)), "set_wait_limit_ns")
+
+
+def workspace_init(workspace, stream=None):
+    """Zero an attention workspace again (after a launch that timed out)."""
+    _need(workspace, "workspace", torch.uint8)
+    _check(library().pkv_workspace_init(workspace.data_ptr(), workspace.numel(),
+                                        _stream(workspace.device, stream)), "workspace_init")
 
 
 def get_device_status(reset=True):

@@ -66,8 +66,10 @@ SIGNATURES = {
         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p,
         ctypes.c_int, ctypes.c_void_p]),
     "pkv_get_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
+    "pkv_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_ulonglong]),
     "pkv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "pkv_abi_version": (ctypes.c_int, []),
+    "pkv_build_hash": (ctypes.c_char_p, []),
 }
 
 
@@ -76,7 +78,9 @@ def lib_path():
 
 
 def load():
-    """Load the CUDA library, building it in-tree first if it is missing.
+    """Load the CUDA library, building it in-tree first if it is missing or
+    was built from sources other than the checkout's (its embedded source
+    hash differs).
 
     There is no fallback: if the library cannot be built or loaded, this raises.
     """
@@ -92,6 +96,10 @@ def load():
             fn = getattr(lib, name)
             fn.restype = res
             fn.argtypes = args
+        want = _build.source_hash()
+        got = lib.pkv_build_hash().decode()
+        if got != want:
+            raise RuntimeError(f"{path} was built from other sources (hash {got}, checkout {want})")
         _lib = lib
         return lib
 

@@ -22,8 +22,10 @@
 namespace pkv {
 
 constexpr unsigned FULL = 0xFFFFFFFFu;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // bounded wait on a stage
-constexpr uint64_t DRAIN_LIMIT_NS = 500000000ull;   // bounded drain after a timeout
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // default bounded wait on a stage
+constexpr uint64_t DRAIN_LIMIT_NS = 500000000ull;   // bounded drain after a timeout (fixed)
+// Per-device limit of the wait on a stage (pkv_set_wait_limit_ns).
+__device__ unsigned long long g_wait_limit_ns = WAIT_LIMIT_NS;
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                                uint32_t b1) {

@@ -9,14 +9,16 @@
 //
 // Decomposition.  Every (sequence, kv head) is a unit of ceil(len/TILE)
 // tiles; units are laid end to end (sequence-major, kv head minor) into one
-// flat space of T tiles, cut into R ranges of equal length.  Without a
-// partition cap R is the number of warps in the grid (one range each); with
-// a cap of C tiles, each warp takes ceil(ceil(T/C)/K) consecutive ranges.
-// A warp streams its tiles with one continuous bulk-copy pipeline that runs
-// across unit and range boundaries, so it never drains between sequences,
-// and every warp gets the same number of tiles whatever the length mix.  A
-// unit inside one range is finished by its warp; a unit cut by range
-// boundaries leaves one partial per range.  Pieces count themselves on a
+// flat space of positions, cut into R ranges of equal length.  A tile takes
+// tc positions and a unit adds a gap after its last tile for its fixed
+// costs (see the layout in the planning below), so equal ranges take about
+// equal time whatever the length mix.  Without a partition cap R is the
+// number of warps in the grid (one range each); with a cap of C tiles
+// (positions are then tiles), each warp takes ceil(ceil(T/C)/K) consecutive
+// ranges.  A warp streams its tiles with one continuous bulk-copy pipeline
+// that runs across unit and range boundaries, so it never drains between
+// sequences.  A unit inside one range is finished by its warp; a unit cut by
+// range boundaries leaves one partial per range.  Pieces count themselves on a
 // ticket; the last one merges them in range order into its own registers
 // (a piece that finds every other piece already counted merges without
 // publishing itself).  Units of more than 8 pieces merge in two levels:
@@ -24,12 +26,13 @@
 // result does not depend on which piece finishes last.
 //
 // Planning.  Every CTA reads the sequence lengths once and scans them into
-// a prefix of tiles per sequence, kept in shared memory (in global memory,
-// written identically by every CTA, for batches of more than PREFIX_SMEM
-// sequences); a warp finds its first tile by binary search and loads its
-// first block ids.  All of this reads only the lengths and the tables and
-// runs before the wait on the previous kernel (programmatic dependent
-// launch); the rest of the kernel runs after it.
+// a prefix of positions per sequence, kept in shared memory (in global
+// memory, written identically by every CTA, for batches of more than
+// PREFIX_SMEM sequences); a warp finds its first tile by binary search and
+// loads its first block ids.  All of this reads only the lengths and the
+// tables and runs before the wait on the previous kernel (programmatic
+// dependent launch); the rest of the kernel runs after it.  A warp that has
+// no tile left to issue lets the next kernel on the stream start launching.
 //
 // Data movement.  Each warp owns a ring of STAGES shared-memory stages.  One
 // lane issues, per stage, TMA tensor loads (cp.async.bulk.tensor, 2-D tensor
@@ -49,10 +52,10 @@
 // Compute.  Tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with
 // the G query heads as the MMA rows; see attn_common.cuh.
 //
-// Faults never trap: waits are bounded (a timeout sets PKV_DEV_TIMEOUT,
-// drains this warp's copies in flight and returns), block ids outside the
-// pool set PKV_DEV_RANGE and are not fetched, lengths above the table's
-// capacity set PKV_DEV_LENGTH and are clamped.
+// Faults never trap: waits are bounded (pkv_set_wait_limit_ns; a timeout
+// sets PKV_DEV_TIMEOUT, drains this warp's copies in flight and returns),
+// block ids outside the pool set PKV_DEV_RANGE and are not fetched, lengths
+// above the table's capacity set PKV_DEV_LENGTH and are clamped.
 #pragma once
 
 #include <cuda.h>
@@ -95,15 +98,44 @@ struct AttnArgs {
 
 constexpr int PREFIX_SMEM = 768;       // sequences whose tile prefix fits in shared memory
 
+// Weights of the position layout: a tile, a unit's start and end, and the
+// expected cost of the unit's end being a piece published mid-stream.
+#ifndef PKV_W_TILE
+#define PKV_W_TILE 8
+#endif
+#ifndef PKV_W_UNIT
+#define PKV_W_UNIT 6
+#endif
+#ifndef PKV_W_PIECE
+#define PKV_W_PIECE 18
+#endif
+
 // R equal ranges over the flat space of T tiles (R <= T, so none is empty).
 struct Sched {
-    long long T, R;
+    long long T, R;                    // positions in the flat space, ranges
     __device__ __forceinline__ long long begin(long long r) const { return r * T / R; }
     // the range holding flat tile t: the largest r with begin(r) <= t
     __device__ __forceinline__ long long range_of(long long t) const { return ((t + 1) * R - 1) / T; }
 };
 
 __device__ __forceinline__ int clamp_len(int len, int cap) { return len > cap ? cap : (len < 0 ? 0 : len); }
+
+// Weights of the position layout (see the planning in the kernel).
+struct Weights {
+    long long tc, uc, pc, lr;          // tile, unit, expected piece; static range length
+};
+
+// Positions taken by one unit of n tiles: its tiles, then a gap for the
+// unit's fixed cost and its expected piece cost.  0 for an empty unit.
+__device__ __forceinline__ long long unit_cost(const Weights& w, long long n) {
+    if (n <= 0) return 0;
+    long long c = n * w.tc + w.uc;
+    if (w.pc) {
+        const long long span = n * w.tc;
+        c += w.pc * (span < w.lr ? span : w.lr) / w.lr;
+    }
+    return c;
+}
 
 template <int D, int G, int BS, int NW, int STAGES>
 struct AttnCfg {
@@ -199,6 +231,8 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
     constexpr int NT = C::NT;
     extern __shared__ unsigned char smem_raw[];
     __shared__ long long s_red[NW];
+    __shared__ Weights s_w;                               // the launch's position weights
+    __shared__ unsigned long long s_wait_limit;           // bounded wait on a stage (ns)
 
     // 1024-byte aligned base (swizzled TMA destinations)
     const uint32_t raw_addr = smem_addr(smem_raw);
@@ -248,11 +282,12 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         long long tot;
         const long long incl = T + block_scan<NT>(v, s_red, &tot) + v;
-        if (s < N) {
-            if (pre_smem) s_prefix[s + 1] = (int)incl;
-            else a.prefix_g[s + 1] = incl;     // every CTA writes the same values
-        }
+        if (s < N && pre_smem) s_prefix[s + 1] = (int)incl;   // (global prefix: positions only, below)
         T += tot;
+    };
+    // clamped length of sequence s (planning and cursor)
+    auto seq_len_raw = [&](int s) -> long long {
+        return lens_smem ? s_len[s] : clamp_len(__ldg(a.seq_lens + s), cap);
     };
     if (pre_smem) {
         // every length this thread scans, loaded before the first scan: one round trip
@@ -277,6 +312,43 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         else a.prefix_g[0] = 0;
     }
     const long long K = a.K;
+    // The position layout.  Units lie in flat order; a tile takes tc
+    // positions and a unit adds uc + its expected piece cost after its last
+    // tile, so ranges of equal length in positions take about equal time.
+    // Measured per warp: a unit boundary costs about 3/4 of a tile, and a
+    // piece published mid-stream (the end of a unit that began in an earlier
+    // range: its publication waits for the warp's memory traffic) about 2 1/4
+    // tiles.  A unit of n tiles is cut by a range boundary with probability
+    // about min(1, n tc / lr), lr the range length, which weights its piece
+    // cost.  Under a partition cap (whose ranges count tiles), and for sizes
+    // whose positions would not fit 32 bits, positions are tiles.
+    Weights wt;
+    wt.tc = 1; wt.uc = 0; wt.pc = 0; wt.lr = 1;
+    if (PKV_W_TILE > 1 && a.cap_tiles == 0 && T > 0 &&
+        T * (PKV_W_TILE + PKV_W_UNIT + PKV_W_PIECE) < (1LL << 30)) {
+        wt.tc = PKV_W_TILE;
+        wt.uc = PKV_W_UNIT;
+        wt.pc = PKV_W_PIECE;
+        wt.lr = T * PKV_W_TILE / K > 1 ? T * PKV_W_TILE / K : 1;
+    }
+    // Prefix of positions per sequence.  In shared memory the tile prefix
+    // already is it when tc = 1; the global prefix (large batches) is written
+    // here only, every CTA writing the same values.
+    if (wt.tc != 1 || !pre_smem) {
+        T = 0;
+        for (int base = 0; base < N; base += NT) {
+            const int s_ = base + tid;
+            const long long n = s_ < N ? (seq_len_raw(s_) + TILE - 1) / TILE : 0;
+            const long long v = (long long)Hkv * unit_cost(wt, n);
+            long long tot;
+            const long long incl = T + block_scan<NT>(v, s_red, &tot) + v;
+            if (s_ < N) {
+                if (pre_smem) s_prefix[s_ + 1] = (int)incl;
+                else a.prefix_g[s_ + 1] = incl;
+            }
+            T += tot;
+        }
+    }
     Sched sc;
     sc.T = T;
     long long rpw = 1;                                    // ranges per warp
@@ -284,39 +356,62 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const long long need = (T + a.cap_tiles - 1) / a.cap_tiles;
         rpw = (need + K - 1) / K;
     }
+    // every range at least one tile long, so each range a unit spans holds
+    // one of its tiles
     sc.R = K * rpw;
-    if (sc.R > T) sc.R = T;
+    if (sc.R > T / wt.tc) sc.R = T / wt.tc;
     if (sc.R > a.R_max) {                                 // cannot happen with a workspace of the queried size
         if (tid == 0 && blockIdx.x == 0) raise_status(PKV_DEV_RANGE);
         sc.R = a.R_max;
     }
+    if (tid == 0) {
+        s_w = wt;
+        s_wait_limit = *(volatile unsigned long long*)&g_wait_limit_ns;
+    }
     __syncthreads();
+    const int tc = (int)wt.tc;
     const long long wg = (long long)blockIdx.x * NW + warp;
     const long long r_first = wg * rpw;
     const long long r_stop = r_first + rpw < sc.R ? r_first + rpw : sc.R;   // this warp's ranges
 
-    // (sequence, kv head, tile) of flat tile f: largest s with prefix[s] <= f
-    auto locate = [&](long long f, int& s_out, int& h_out, int& t_out) {
-        int lo = 0, hi = N - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            const long long pm = pre_smem ? (long long)s_prefix[mid] : a.prefix_g[mid];
-            if (pm <= f) lo = mid; else hi = mid - 1;
+    // The first tile at or after position `pos`: its (sequence, kv head,
+    // tile) and position, or -1 when there is none.
+    auto locate = [&](long long pos, int& s_out, int& h_out, int& t_out) -> long long {
+#pragma unroll 1
+        for (int it = 0; it < 2; ++it) {
+            if (pos >= sc.T) return -1;
+            int lo = 0, hi = N - 1;                       // largest s with prefix[s] <= pos
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                const long long pm = pre_smem ? (long long)s_prefix[mid] : a.prefix_g[mid];
+                if (pm <= pos) lo = mid; else hi = mid - 1;
+            }
+            const long long p0 = pre_smem ? (long long)s_prefix[lo] : a.prefix_g[lo];
+            const long long n = (seq_len_raw(lo) + TILE - 1) / TILE;
+            const long long ucs = unit_cost(s_w, n);
+            const long long off = pos - p0;
+            long long h = off / ucs;
+            const long long t = (off - h * ucs + tc - 1) / tc;
+            if (t < n) {
+                s_out = lo; h_out = (int)h; t_out = (int)t;
+                return p0 + h * ucs + t * tc;
+            }
+            if (++h < Hkv) {                              // in the unit's end gap: the next unit
+                s_out = lo; h_out = (int)h; t_out = 0;
+                return p0 + h * ucs;
+            }
+            pos = pre_smem ? (long long)s_prefix[lo + 1] : a.prefix_g[lo + 1];   // the next sequence
         }
-        const long long p0 = pre_smem ? (long long)s_prefix[lo] : a.prefix_g[lo];
-        const long long p1 = pre_smem ? (long long)s_prefix[lo + 1] : a.prefix_g[lo + 1];
-        const long long nt = (p1 - p0) / Hkv;
-        const long long off = f - p0;
-        s_out = lo;
-        h_out = (int)(off / nt);
-        t_out = (int)(off % nt);
+        return -1;
     };
 
     const uint64_t pol_stream = policy_evict_first();
 
     // ---- producer cursor (every lane keeps an identical copy) ------------------
     long long r = r_first;                                // range of the next tile to issue
-    long long f = 0, f_end = 0, f_stop = 0;
+    long long f = 0, f_end = 0, f_stop = 0;             // positions: next tile, range end, warp's end
+    long long pnext = 0;                                  // position of the next unit's tile 0
+    int puc = 1;                                          // positions a unit of this sequence takes
     int ps = 0, ph = 0, pt = 0, plen = 0, pnt = 0, next_len = 0;
     int pcow = -1, next_cow = -1;                         // copy-on-write source of ps, ps + 1
     bool range_first = true;
@@ -334,7 +429,11 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
     auto cow_of = [&](int s) -> int { return (a.cow_src && s < N) ? __ldg(a.cow_src + s) : -1; };
     auto advance_unit = [&]() {
         pt = 0;
-        if (++ph < Hkv) return;
+        f = pnext;                                        // (empty sequences take no positions)
+        if (++ph < Hkv) {
+            pnext += puc;
+            return;
+        }
         ph = 0;
         ++ps;
         plen = next_len;
@@ -348,6 +447,8 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         next_len = seq_len(ps + 1);
         next_cow = cow_of(ps + 1);
+        puc = (int)unit_cost(s_w, pnt);
+        pnext = f + puc;
     };
     // Block ids of the current tile's batch of 32 logical blocks (one per
     // lane), taken from the prefetched batch when it holds them; then the
@@ -369,18 +470,23 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
             pre_seq = ps + 1; pre_base = 0; pre = load_batch(ps + 1, 0, next_len);
         }
     };
-    const bool have_work = r_first < r_stop;
-    if (have_work) {
-        f = sc.begin(r_first);
+    bool have_work = false;
+    if (r_first < r_stop) {
         f_end = sc.begin(r_first + 1);
         f_stop = sc.begin(r_stop);
-        locate(f, ps, ph, pt);
-        plen = seq_len(ps);
-        pnt = (plen + TILE - 1) / TILE;
-        next_len = seq_len(ps + 1);
-        pcow = cow_of(ps);
-        next_cow = cow_of(ps + 1);
-        fetch_ids(pt * C::BPT);                           // the first tile's block ids
+        const long long fpos = locate(sc.begin(r_first), ps, ph, pt);
+        if (fpos >= 0 && fpos < f_stop) {                 // (a range in a unit's end gap has no tile)
+            have_work = true;
+            f = fpos;
+            plen = seq_len(ps);
+            pnt = (plen + TILE - 1) / TILE;
+            puc = (int)unit_cost(s_w, pnt);
+            pnext = fpos - (long long)pt * tc + puc;
+            next_len = seq_len(ps + 1);
+            pcow = cow_of(ps);
+            next_cow = cow_of(ps + 1);
+            fetch_ids(pt * C::BPT);                       // the first tile's block ids
+        }
     }
 
     // Everything so far read only the lengths and the block tables, which no
@@ -399,18 +505,20 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     // Stage the next tile into stage `st`; false when this warp has no more tiles.
     auto issue = [&](int st) -> bool {
-        if (f == f_stop) return false;
-        if (f == f_end) {                                 // next range of this warp (contiguous)
+        if (f >= f_stop) return false;
+        if (f >= f_end) {                                 // next range of this warp (contiguous)
             ++r;
             f_end = sc.begin(r + 1);
             range_first = true;
         }
+        // position of the tile after this one
+        const long long f_next = pt + 1 < pnt ? f + tc : pnext;
         const int nv = min(TILE, plen - pt * TILE);
         int flags = 0;
         if (pt == 0) flags |= F_UNIT_START;
         if (pt == pnt - 1) flags |= F_UNIT_END;
         if (range_first || pt == 0) flags |= F_FIRST;
-        if (f + 1 == f_end || pt == pnt - 1) flags |= F_LAST;
+        if (f_next >= f_end || pt == pnt - 1) flags |= F_LAST;
         range_first = false;
         const int lb0 = pt * C::BPT;
         fetch_ids(lb0);
@@ -431,7 +539,7 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 uint16_t* dv = nullptr;
                 uint16_t* ck = nullptr;
                 uint16_t* cv = nullptr;
-                if (nblk >= 0 && nblk < a.num_blocks) {
+                if (nblk >= 0 && nblk < a.num_blocks && pcow != PKV_COW_NO_APPEND) {
                     const size_t brow = (size_t)(a.row_base + ((long long)nblk * Hkv + ph) * BS);
                     dk = a.k_pool + (brow + (plen - 1) % BS) * D;
                     dv = a.v_pool + (brow + (plen - 1) % BS) * D;
@@ -453,7 +561,7 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const uint32_t dV = dK + C::KT_BYTES;
             uint32_t bytes = (flags & F_FIRST) ? C::Q_BYTES : 0u;
             // fused append: the unit's last tile also brings the new token's rows
-            const bool app = fused_append && (flags & F_UNIT_END);
+            const bool app = fused_append && (flags & F_UNIT_END) && pcow != PKV_COW_NO_APPEND;
             if (app) bytes += 4u * D;
             bool bad = false;
 #pragma unroll
@@ -490,8 +598,8 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 }
             }
         }
-        ++f;
         if (++pt == pnt) advance_unit();
+        else f += tc;
         return true;
     };
 
@@ -526,9 +634,9 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
             return;
         }
         const long long nt = (m.len + TILE - 1) / TILE;
-        const long long au = m.f - m.t;                    // the unit's first flat tile
+        const long long au = m.f - (long long)m.t * tc;   // position of the unit's tile 0
         const long long r_lo = sc.range_of(au);
-        const long long r_hi = sc.range_of(au + nt - 1);
+        const long long r_hi = sc.range_of(au + (nt - 1) * tc);
         // partial slot of range j: 0 if the unit began in an earlier range
         auto piece_row = [&](long long j) -> size_t {
             return ((size_t)j * 2 + ((au < sc.begin(j)) ? 0 : 1)) * G + g_row;
@@ -674,17 +782,29 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
     };
 
     // ---- main loop ------------------------------------------------------------------
+    // The next kernel on the stream may start launching once every warp has no
+    // tile left to issue: its CTAs become resident as this grid's CTAs exit
+    // and plan while the last tiles here finish; they touch no data before
+    // their wait on this grid's completion.
+    bool released = false;
+    auto release = [&]() {
+        if (!released) {
+            pdl_launch_dependents();
+            released = true;
+        }
+    };
     int issued = 0;
     bool more = have_work;
     while (issued < STAGES && more) {
         more = issue(issued);
         if (more) ++issued;
     }
+    if (!more) release();
     int failed_at = -1;
     for (int i = 0; i < issued; ++i) {
         const int st = i % STAGES;
         const bool ok = mbar_wait_bounded(smem_addr(&bars[st]), (uint32_t)(i / STAGES) & 1u,
-                                          WAIT_LIMIT_NS);
+                                          s_wait_limit);
         if (__any_sync(FULL, !ok)) { failed_at = i; break; }
         const StageMeta m = meta[st];
         unsigned char* sKp = ring + (size_t)st * C::STAGE_BYTES;
@@ -750,12 +870,10 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (more) {
             more = issue(st);
             if (more) ++issued;
+            else release();
         }
     }
-    // Let the next kernel on the stream start launching only now: its CTAs
-    // would otherwise sit resident (waiting) beside this kernel's warps for
-    // the whole launch.
-    pdl_launch_dependents();
+    release();                                            // (a warp that stopped early)
     if (failed_at >= 0) {
         if (lane == 0) raise_status(PKV_DEV_TIMEOUT);
         for (int i = failed_at; i < issued; ++i)

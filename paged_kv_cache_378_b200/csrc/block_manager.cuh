@@ -17,6 +17,10 @@
 //     head + k (an exclusive scan of "takes a block" over the writers);
 //   - copy pairs are numbered by an exclusive scan of "copies".
 // One CTA of 1024 threads; writer i is handled by thread i mod 1024.
+//
+// An abort (free blocks short, an index out of range) changes no state and
+// leaves outputs that make a step queued behind it harmless: every slot -1,
+// no copy pair, and cow_src = PKV_COW_NO_APPEND for every sequence.
 #pragma once
 
 #include "pkv_device.cuh"
@@ -138,8 +142,29 @@ __global__ void __launch_bounds__(BM_THREADS, 1) block_manager_kernel(const BmAr
         total_copies += c;
     }
     const int head = a.free_state[0], avail = a.free_state[1];
-    if (s_abort || total_takes > avail) {               // change nothing
+    // the blocks the takers will get, checked before anything changes
+    int newb[BM_PER_THREAD];
+#pragma unroll
+    for (int k = 0; k < BM_PER_THREAD; ++k) newb[k] = -1;
+    if (total_takes <= avail) {
+#pragma unroll
+        for (int k = 0; k < BM_PER_THREAD; ++k) {
+            if (seq[k] < 0 || !takes[k]) continue;
+            newb[k] = a.free_ring[(head + take_base[k]) % a.num_blocks];
+            if (newb[k] < 0 || newb[k] >= a.num_blocks) { raise_status(PKV_DEV_RANGE); atomicExch(&s_abort, 1); }
+        }
+    }
+    __syncthreads();
+    if (s_abort || total_takes > avail) {
+        // Change nothing, and say so to whatever is queued behind this step:
+        // no slot (kv_append skips slot -1), no copy pair, and per sequence
+        // the marker that makes the fused append + attention append nothing.
         if (tid == 0 && total_takes > avail) raise_status(PKV_DEV_NOBLOCKS);
+        for (int i = tid; i < N; i += BM_THREADS) {
+            a.slot_mapping[i] = -1;
+            if (a.cow_src) a.cow_src[i] = PKV_COW_NO_APPEND;
+        }
+        if (tid == 0) *a.num_pairs = 0;
         return;
     }
     __syncthreads();                                    // every count read before any is changed
@@ -150,8 +175,7 @@ __global__ void __launch_bounds__(BM_THREADS, 1) block_manager_kernel(const BmAr
         const int s = seq[k], p = pos[k];
         int32_t* entry = a.block_tables + (size_t)s * a.max_blocks + p / B;
         if (takes[k]) {
-            const int nb = a.free_ring[(head + take_base[k]) % a.num_blocks];
-            if (nb < 0 || nb >= a.num_blocks) { raise_status(PKV_DEV_RANGE); continue; }
+            const int nb = newb[k];
             a.refcount[nb] = 1;
             if (copies[k]) {
                 const int tail = s_tail[k * BM_THREADS + tid];

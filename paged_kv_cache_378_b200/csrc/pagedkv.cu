@@ -136,6 +136,15 @@ bool fill_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, 
     return true;
 }
 
+// Upper bound on the ranges of one launch over a grid of K warps (see the
+// planning in the attention kernel): K ranges, or at most ceil(T / cap) + K
+// under a cap of cap_tiles, for T <= max_tiles_total.
+long long ranges_bound(long long K, long long max_tiles_total, int cap_tiles) {
+    long long r = K;
+    if (cap_tiles > 0) r += (max_tiles_total + cap_tiles - 1) / cap_tiles + 1;
+    return r;
+}
+
 int grid_warps_for(int D, int G, int BS);
 
 // The tile prefix of large batches, two partials per range (one range per
@@ -151,10 +160,9 @@ bool workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_
     if (pt < 0) return false;
     const int tile = tile_tokens(head_dim, block_size);
     const long long max_tiles = ((long long)max_blocks * block_size + tile - 1) / tile;
-    long long r_max = grid_warps_for(head_dim, num_q_heads / num_kv_heads, block_size);
+    const long long K = grid_warps_for(head_dim, num_q_heads / num_kv_heads, block_size);
     const int cap_tiles = pt / tile;
-    if (cap_tiles > 0)
-        r_max += ((long long)num_seqs * num_kv_heads * max_tiles + cap_tiles - 1) / cap_tiles + 1;
+    const long long r_max = ranges_bound(K, (long long)num_seqs * num_kv_heads * max_tiles, cap_tiles);
     return fill_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, r_max, cap_tiles, w);
 }
 
@@ -278,11 +286,10 @@ bool noalloc_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
     if (pt < 0) return false;
     const int tile = tile_tokens(head_dim, block_size);
     const long long max_tiles = ((long long)max_blocks * block_size + tile - 1) / tile;
-    long long r_cap = 0;
+    const long long tiles = (long long)num_seqs * num_kv_heads * max_tiles;
     const int cap_tiles = pt / tile;
-    if (cap_tiles > 0)
-        r_cap = ((long long)num_seqs * num_kv_heads * max_tiles + cap_tiles - 1) / cap_tiles + 1;
-    return fill_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, grid_warps + r_cap, cap_tiles, w);
+    return fill_layout(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                       ranges_bound(grid_warps, tiles, cap_tiles), cap_tiles, w);
 }
 
 // Device address of the scratch on the current device (set up on first use).
@@ -399,9 +406,17 @@ const void* host_pool_device_ptr(const void* p) {
 
 }  // namespace
 
+#ifndef PKV_BUILD_HASH
+#define PKV_BUILD_HASH "0000000000000000"
+#endif
+// The build's source hash, after a tag the loader finds in the file itself.
+__attribute__((used)) static const char kBuildTag[] = "PKV_BUILD_HASH:" PKV_BUILD_HASH;
+
 extern "C" {
 
 int pkv_abi_version(void) { return PKV_ABI_VERSION; }
+
+const char* pkv_build_hash(void) { return kBuildTag + sizeof("PKV_BUILD_HASH:") - 1; }
 
 const char* pkv_strerror(int code) {
     switch (code) {
@@ -492,6 +507,9 @@ int pkv_prefix_block_hashes(const int32_t* tokens, int max_tokens, const int32_t
                             const uint64_t* parent_hashes, int num_seqs, int block_size,
                             uint64_t* hashes, int max_blocks, void* stream) {
     if (num_seqs < 0 || max_tokens < 0 || max_blocks < 0 || block_size <= 0) return PKV_ERR_SHAPE;
+    // resuming needs the stored hash of the block before: without it the
+    // chain would restart from 0 and match another sequence's first blocks
+    if (first_block && !parent_hashes) return PKV_ERR_NULL;
     if (num_seqs == 0 || max_blocks == 0) return PKV_OK;
     if (!tokens || !seq_lens || !hashes) return PKV_ERR_NULL;
     const int per_cta = 8;                                  // warps (sequences) per CTA
@@ -642,6 +660,12 @@ int pkv_paged_decode_attention_noalloc(const pkv_cache_t* cache, int layer, cons
     return with_instance(D, G, BS, [&](auto inst) {
         return decltype(inst)::launch(mk, mv, a, grid_warps / kAttnWarps, s);
     });
+}
+
+int pkv_set_wait_limit_ns(unsigned long long limit_ns) {
+    const unsigned long long v = limit_ns ? limit_ns : pkv::WAIT_LIMIT_NS;
+    if (cudaMemcpyToSymbol(pkv::g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) return PKV_ERR_CUDA;
+    return PKV_OK;
 }
 
 int pkv_get_device_status(unsigned int* status_out, int reset) {

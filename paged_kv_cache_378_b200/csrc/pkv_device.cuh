@@ -64,10 +64,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of the same phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 // Wait for phase `parity` of the barrier to complete, giving up after
 // `limit_ns` nanoseconds.  Returns false on timeout (the caller records it).
+// try_wait may suspend the thread until the phase completes (up to a
+// hardware time limit), so a limit under a microsecond polls with the
+// non-blocking test instead and lets the clock decide.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   uint64_t limit_ns) {
+    if (limit_ns < 1000) {
+        const uint64_t t0 = global_timer_ns();
+#pragma unroll 1
+        while (true) {
+            if (mbar_test_wait(bar, parity)) return true;
+            if (global_timer_ns() - t0 > limit_ns) return false;
+        }
+    }
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
         if (mbar_try_wait(bar, parity)) return true;
@@ -78,6 +100,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
         if (global_timer_ns() - t0 > limit_ns) return false;
     }
 }
+
 
 // ---- bulk copy global -> shared (non-tensor TMA) ---------------------------
 
@@ -113,6 +136,15 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+// atomic add at gpu scope with acquire-release order: the writes this thread
+// made or saw before it (cumulatively: a warp's writes ordered before it by
+// the warp's barrier) are visible to whoever reads the new value with
+// acquire, and writes seen by the previous releasers are visible after it
+__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
 }
 __device__ __forceinline__ int ld_cg(const int* p) {
     int v;

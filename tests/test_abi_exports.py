@@ -35,6 +35,16 @@ def test_library_loads_and_exports_every_declared_symbol():
     assert set(_declared()) <= exported
 
 
+def test_library_is_built_from_these_sources():
+    # the loaded library carries the hash of the checkout's sources, header
+    # and flags, both in its exported string and in the file the loader scans
+    from paged_kv_cache_378_b200 import build as b
+    lib = pkv.library()
+    assert lib.pkv_build_hash().decode() == b.source_hash()
+    assert b.built_hash(_lib.lib_path()) == b.source_hash()
+    assert not b.needs_build(_lib.lib_path())
+
+
 def test_version_and_error_strings():
     lib = pkv.library()
     assert lib.pkv_abi_version() == 1
@@ -104,6 +114,10 @@ def test_host_argument_checks_before_launch():
     assert sw(P(c), P(_cache(num_blocks=3)), 16, 0, 0, None) == 0
     assert sw(P(c), P(_cache(num_blocks=3)), None, 2, 1, None) == -1
     assert sw(P(c), P(_cache(k_pool=0)), 16, 1, 0, None) == -1
+    # prefix hashes: resuming (first_block) needs the parent hashes
+    ph = lib.pkv_prefix_block_hashes
+    assert ph(16, 64, 16, None, 16, None, 4, 16, 16, 4, None) == -1
+    assert ph(16, 64, 16, None, None, None, 0, 16, 16, 4, None) == 0
     # device block manager step: state required, sizes checked, at most 4096 sequences
     st = _lib.PkvBlockState(16, 16, 16, 16, 16)
     bm = lib.pkv_block_manager_step

@@ -256,3 +256,48 @@ def test_device_step_with_copy_on_write_folded_into_attention():
     lens = np.array([bm.lengths[s] for s in writers], np.int32)
     ref = oa.paged_decode_attention(u16(q), ek, ev, tables, lens, B, D ** -0.5)
     assert_close(f64(out), ref, "copy-on-write folded into attention")
+
+
+def test_aborted_step_leaves_a_chained_device_step_harmless():
+    # Free blocks run short: the manager changes no state and writes outputs
+    # that make what is already queued behind it do nothing -- slots -1, no
+    # copy pair, cow_src = COW_NO_APPEND -- so a device-only step chained on
+    # the same stream (block copy with the device count, kv_append, fused
+    # append + attention with cow_src) leaves both pools byte-identical.
+    from .stepping import u16
+    rng = np.random.default_rng(5)
+    B, H, D, G, NB = 16, 2, 64, 4, 16
+    bm = BlockManager(NB, B, free_order=rng.permutation(NB))
+    bm.add_sequence(0, 37)             # 3 blocks, shared tail below: 3 copies needed
+    for c in range(1, 4):
+        bm.fork(0, c)
+    for s in range(4, 8):
+        bm.add_sequence(s, 32)         # full tails: 4 more blocks needed
+    assert len(bm.free) == 5           # 7 needed
+    writers = list(range(8))
+    st = _snapshot(bm, writers, 4)
+    before = [t.clone() for t in (st.block_tables, st.seq_lens, st.refcount, st.free_ring,
+                                  st.free_state)]
+    g = torch.Generator().manual_seed(5)
+    kd = torch.randn((1, NB, H, B, D), generator=g).to(torch.bfloat16).cuda()
+    vd = torch.randn((1, NB, H, B, D), generator=g).to(torch.bfloat16).cuda()
+    k0, v0 = u16(kd), u16(vd)
+    q = torch.randn((8, H * G, D), generator=g).to(torch.bfloat16).cuda()
+    kn = torch.randn((8, H, D), generator=g).to(torch.bfloat16).cuda()
+    vn = torch.randn((8, H, D), generator=g).to(torch.bfloat16).cuda()
+    slots, pairs, npairs, cow = pkv.block_manager_step(st, B, with_cow_src=True)
+    pkv.block_copy(pairs, kd, vd, num_pairs=npairs)
+    pkv.kv_append(kn, vn, slots, kd, vd)
+    out = torch.empty_like(q)
+    ws = pkv.make_workspace(8, H * G, H, D, 4, B, 0)
+    pkv.append_paged_decode_attention(kn, vn, q, kd, vd, st.block_tables, st.seq_lens, B,
+                                      D ** -0.5, out, workspace=ws, cow_src=cow)
+    torch.cuda.synchronize()
+    assert pkv.get_device_status(reset=True) == pkv.DEV_NOBLOCKS
+    assert slots.cpu().tolist() == [-1] * 8
+    assert int(npairs.item()) == 0
+    assert cow.cpu().tolist() == [pkv.COW_NO_APPEND] * 8
+    assert np.array_equal(u16(kd), k0) and np.array_equal(u16(vd), v0)
+    after = (st.block_tables, st.seq_lens, st.refcount, st.free_ring, st.free_state)
+    for a, b in zip(before, after):
+        assert torch.equal(a, b)
