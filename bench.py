@@ -42,6 +42,7 @@ METRIC = "paged decode attention KV GB/s and % of HBM peak; decode tokens/s per 
 UNIT = "GB/s"
 DEFAULT_WORKLOAD = "continuous_batch"
 FALLBACK_HBM_GBS = 6650.0
+SPIN_CYCLES = 4_000_000    # ~2 ms of spinning ahead of a timed region
 NOMINAL_HBM_GBS = 8000.0   # the ~8 TB/s the 70 % bandwidth target is stated against
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "attention_traffic.json")
 EVENT_EVERY = 8            # attention events on every 8th timed step
@@ -973,6 +974,7 @@ def measure_config(pkv, key, B, part, device, sampler, peak, peak_kind, min_regi
     steps = max(20, int(math.ceil(min_region_s * 1e3 / max(est, 1e-3))))
     torch.cuda.synchronize(device)
     wall0 = time.time()
+    torch.cuda._sleep(SPIN_CYCLES)
     ms = region_ms(gs, steps, 8)
     wall1 = time.time()
     stats = launch_stats(gs, max(8, min(200, int(math.ceil(200 / spec.num_layers)))), 8 + steps)
@@ -1048,14 +1050,9 @@ def main():
     part = spec.partition_tokens if args.partition < 0 else args.partition
     seed = rank_seed(spec.seed, rank)
 
-    # cpu baseline first, before this process touches the GPU (its pool is
-    # spawned; rank 0 at N = 1 only)
     w_meta = make_workload(args.workload, block_size=B, seed=seed, values=False)
     unique_bytes = w_meta.unique_kv_bytes_read()
     logical_bytes = w_meta.kv_bytes_read()
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(args.workload, B, seed, unique_bytes)
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
@@ -1107,6 +1104,10 @@ def main():
         dist.barrier()
     torch.cuda.synchronize(device)
     wall0 = time.time()
+    # A spin kernel ahead of the region keeps the GPU busy while the host
+    # enqueues the steps, so the events time the device, not the host's
+    # first enqueue latency (a short region would otherwise include it).
+    torch.cuda._sleep(SPIN_CYCLES)
     t_start.record(gs.stream)
     nl = spec.num_layers
     fast = gs.prepared()
@@ -1192,6 +1193,12 @@ def main():
             per_config.append(measure_config(pkv, key, bs, sp.partition_tokens if p < 0 else p,
                                              device, sampler, peak, peak_kind))
     sampler.stop()
+
+    # the oracle on the host cores last: a spawned pool, so starting it after
+    # this process used the GPU is safe (rank 0 at N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, B, seed, unique_bytes)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -18,10 +18,18 @@ import pytest
 import torch
 
 from workload import make_workload
+from workload.configs import WorkloadSpec
 
 from .stepping import assert_close, f64
 
 pytestmark = pytest.mark.gpu
+
+
+# More than 768 sequences (the tile prefix then lives in the scratch too), the
+# widest group (G = 8) at head_dim 128: the largest scratch of an uncapped call.
+WIDE = WorkloadSpec(key="noalloc_wide", title="1000 seqs, G=8, d128", num_layers=1, num_seqs=1000,
+                    num_q_heads=32, num_kv_heads=4, head_dim=128, block_size=16, seed=77,
+                    lengths="uniform:1,300")
 
 
 def _inputs(key, device):
@@ -37,7 +45,7 @@ def _inputs(key, device):
     return w, spec, kp, vp, q, tables, lens
 
 
-@pytest.mark.parametrize("key", ["continuous_batch", "long_context"])
+@pytest.mark.parametrize("key", ["continuous_batch", "long_context", WIDE])
 def test_noalloc_matches_workspace_call_on_two_calls(key):
     import paged_kv_cache_378_b200 as pkv
     from paged_kv_cache_378_b200._lib import PkvCache
@@ -52,6 +60,8 @@ def test_noalloc_matches_workspace_call_on_two_calls(key):
     ref = torch.empty_like(q)
     ws = pkv.make_workspace(w.num_seqs, spec.num_q_heads, spec.num_kv_heads, spec.head_dim,
                             w.max_blocks, w.block_size, 0, device=dev)
+    # the scratch holds what the workspace-taking call needs for the same sizes
+    assert ws.numel() <= 16 << 20, ws.numel()
     pkv.paged_decode_attention(q, kp, vp, tables, lens, w.block_size, spec.scale, ref, workspace=ws)
     torch.cuda.synchronize()
 
@@ -71,7 +81,10 @@ def test_noalloc_matches_workspace_call_on_two_calls(key):
     want = f64(ref)
     assert np.all(np.isfinite(want))
     for i, out in enumerate(outs):
-        assert_close(f64(out), want, f"{key} no-alloc call {i}")
+        name = key if isinstance(key, str) else key.key
+        assert_close(f64(out), want, f"{name} no-alloc call {i}")
+        # same kernel, same schedule: the same bits
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), f"{name} call {i}"
 
 
 def test_noalloc_refuses_requests_larger_than_its_scratch():
