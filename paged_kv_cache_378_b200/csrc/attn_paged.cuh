@@ -681,25 +681,12 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
             auto slot_of = [&](long long e) -> size_t { return slot_of_level(e, groups); };
             const unsigned others = (unsigned)(last - first);
             unsigned seen = 0;
-#if PKV_X_PRECHECK
-            // only the first element is likely to finish last (it ends its
-            // warp's range; the others start theirs): only it checks first
-            if (mine == first) {
-                if (lane == 0) seen = ld_acquire(ticket);
-                seen = __shfl_sync(FULL, seen, 0);
-            }
-#else
             if (lane == 0) seen = ld_acquire(ticket);
             seen = __shfl_sync(FULL, seen, 0);
-#endif
             bool stored = false;
             if (seen != others) {
                 store_state(slot_of(mine));
-#if PKV_X_FENCE
-                if (g_row < G) __threadfence();             // the lanes that stored
-#else
                 __threadfence();
-#endif
                 __syncwarp();
                 unsigned prev = 0;
                 if (lane == 0) prev = atomicAdd(ticket, 1u);
