@@ -78,9 +78,10 @@ def load_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def load_traffic(workload_key, block_size, step):
+def load_traffic(workload_key, block_size, step, partition):
     """DRAM bytes per attention launch from the committed ncu summary, or None
-    if absent, for another workload or step, or taken on different kernel source."""
+    if absent, for another workload, step or partition cap, or taken on
+    different kernel source."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             rec = json.load(f)
@@ -89,6 +90,7 @@ def load_traffic(workload_key, block_size, step):
     for r in rec.get("captures", []):
         if r.get("workload") == workload_key and int(r.get("block_size", -1)) == block_size \
                 and r.get("step") == step \
+                and int(r.get("partition_tokens", 0)) == partition \
                 and r.get("kernel_source_hash") == kernel_source_hash():
             return r.get("dram_bytes_per_launch")
     return None
@@ -463,6 +465,62 @@ def block_manager_timing(pkv, w, device, iters=100):
     if pkv.get_device_status(reset=True):
         raise SystemExit("device status raised by the block manager step")
     return sum(a.elapsed_time(b) for a, b in evs) / iters * 1e3
+
+
+def block_manager_chained_timing(pkv, w, gs, device, steps=40, chunks=10):
+    """Device time the block-manager step adds when it runs between chained
+    attention launches (the device-only decode loop), against the launches
+    alone: median over chunks of `steps` steps.  The step works on its own
+    copy of the pre-step state (tables with spare columns so no sequence
+    outgrows them), restored before every chunk; the attention launches read
+    the workload's own inputs, so their work is the same in both."""
+    from paged_kv_cache_378_b200._lib import PkvBlockState
+    st = prestep_state(w)
+    bt = st["block_tables"]
+    st["block_tables"] = np.concatenate([bt, np.full((bt.shape[0], 16), -1, bt.dtype)], axis=1)
+    pristine = {k: torch.from_numpy(np.ascontiguousarray(v)).to(device) for k, v in st.items()}
+    live = {k: v.clone() for k, v in pristine.items()}
+    c = PkvBlockState(live["block_tables"].data_ptr(), live["seq_lens"].data_ptr(),
+                      live["refcount"].data_ptr(), live["free_ring"].data_ptr(),
+                      live["free_state"].data_ptr())
+    N, maxb = live["block_tables"].shape
+    order = None
+    if w.batch_order is not None:
+        order = torch.from_numpy(np.ascontiguousarray(w.batch_order, dtype=np.int32)).to(device)
+    slots = torch.empty(N, dtype=torch.int64, device=device)
+    pairs = torch.empty((N, 2), dtype=torch.int32, device=device)
+    npairs = torch.zeros(1, dtype=torch.int32, device=device)
+    cow = torch.empty(N, dtype=torch.int32, device=device)
+    lib = pkv.library()
+    args = (ctypes.byref(c), N, maxb, int(w.num_blocks), int(w.block_size),
+            ctypes.c_void_p(order.data_ptr()) if order is not None else None,
+            ctypes.c_void_p(slots.data_ptr()), ctypes.c_void_p(pairs.data_ptr()),
+            ctypes.c_void_p(npairs.data_ptr()), ctypes.c_void_p(cow.data_ptr()), gs.sp)
+    launch = gs.prepared()
+
+    def chunk(with_step):
+        for k in live:
+            live[k].copy_(pristine[k])
+        torch.cuda._sleep(SPIN_CYCLES)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(gs.stream)
+        for i in range(steps):
+            launch(i)
+            if with_step and lib.pkv_block_manager_step(*args):
+                raise SystemExit("block manager step refused its arguments")
+        e1.record(gs.stream)
+        torch.cuda.synchronize(device)
+        return e0.elapsed_time(e1) / steps * 1e3
+
+    for _ in range(2):
+        chunk(True)
+        chunk(False)
+    alone = float(np.median([chunk(False) for _ in range(chunks)]))
+    both = float(np.median([chunk(True) for _ in range(chunks)]))
+    if pkv.get_device_status(reset=True):
+        raise SystemExit("device status raised by the chained block manager steps")
+    return alone, both
 
 
 def prefix_hash_timing(pkv, w, device, iters=50):
@@ -1167,6 +1225,8 @@ def main():
     extras = {}
     if not args.no_extras:
         bm_us = block_manager_timing(pkv, w, device) if w.num_seqs <= 4096 else None
+        bm_chain = (block_manager_chained_timing(pkv, w, gs, device)
+                    if bm_us is not None and spec.num_layers == 1 else None)
         extras["swap"] = swap_timing(pkv, w, device)
         extras["prefix_hash"] = prefix_hash_timing(pkv, w, device)
         extras["prefix_hash_decode"] = prefix_hash_decode_timing(pkv, w, device)
@@ -1174,11 +1234,19 @@ def main():
             "us_per_step": bm_us, "num_seqs": w.num_seqs,
             "what": "device block-manager step (slot mapping, copy-on-write decisions, block "
                     "allocation) timed alone on this step's pre-step state, restored between launches"}
+        if bm_chain is not None:
+            extras["block_manager"].update({
+                "chained_attention_us": bm_chain[0], "chained_with_step_us": bm_chain[1],
+                "added_between_chained_launches_us": bm_chain[1] - bm_chain[0],
+                "chained_what": "attention launches chained back to back, with and without the "
+                                "step between them (it reads and decides before its wait on the "
+                                "previous launch, so only its writes and the next launch's start "
+                                "are added)"})
 
     peak, peak_kind = load_peak()
     alg = algorithmic_bytes(w, spec, B, gs, unique_bytes)
     achieved = alg["total"] / (attn_avg_ms * 1e-3) / 1e9
-    traffic = load_traffic(args.workload, B, gs.mode)
+    traffic = load_traffic(args.workload, B, gs.mode, gs.partition)
     launches_per_step = gs.launches_per_step
     del gs, replicas, w
     torch.cuda.empty_cache()

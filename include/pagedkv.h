@@ -256,8 +256,13 @@ typedef struct pkv_block_state {
  * entry -1 (pkv_kv_append skips it), *num_pairs = 0 (no copy), and, when
  * cow_src is given, cow_src[s] = PKV_COW_NO_APPEND for every sequence (the
  * fused pkv_append_paged_decode_attention then appends and copies nothing).
- * The kernel does not release its dependents early, so an attention launch
- * that follows on the stream reads the new lengths.
+ * The kernel reads all of its state (order, lengths, tables, counts, free
+ * ring and state) and makes every decision before its wait on the previous
+ * kernel, and writes only after it; so that state, like the attention
+ * calls' lengths and tables, must be written by copies or by kernels that
+ * do not release their dependents early (in this library only this kernel
+ * writes it).  It does not release its own dependents early, so an attention
+ * launch that follows on the stream reads the new lengths.
  */
 int pkv_block_manager_step(const pkv_block_state_t* state, int num_seqs,
                            int max_blocks_per_seq, int num_blocks, int block_size,

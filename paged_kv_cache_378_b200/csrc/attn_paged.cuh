@@ -104,7 +104,7 @@ constexpr int PREFIX_SMEM = 768;       // sequences whose tile prefix fits in sh
 #define PKV_W_TILE 8
 #endif
 #ifndef PKV_W_UNIT
-#define PKV_W_UNIT 6
+#define PKV_W_UNIT 10
 #endif
 #ifndef PKV_W_PIECE
 #define PKV_W_PIECE 18
@@ -315,13 +315,14 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // The position layout.  Units lie in flat order; a tile takes tc
     // positions and a unit adds uc + its expected piece cost after its last
     // tile, so ranges of equal length in positions take about equal time.
-    // Measured per warp: a unit boundary costs about 3/4 of a tile, and a
-    // piece published mid-stream (the end of a unit that began in an earlier
-    // range: its publication waits for the warp's memory traffic) about 2 1/4
-    // tiles.  A unit of n tiles is cut by a range boundary with probability
-    // about min(1, n tc / lr), lr the range length, which weights its piece
-    // cost.  Under a partition cap (whose ranges count tiles), and for sizes
-    // whose positions would not fit 32 bits, positions are tiles.
+    // Timed per warp: a unit's fixed costs (its query load, state reset and
+    // finish) come to about one tile, and a piece of a split unit (published,
+    // counted, possibly merged) about two more.  A unit of n tiles is cut by a
+    // range boundary with probability about min(1, n tc / lr), lr the range
+    // length, which weights its piece cost.  The weights (tile 8, unit 10,
+    // piece 18) are the best of a sweep timed on the length mixes of the
+    // benchmark workloads.  Under a partition cap (whose ranges count tiles),
+    // and for sizes whose positions would not fit 32 bits, positions are tiles.
     Weights wt;
     wt.tc = 1; wt.uc = 0; wt.pc = 0; wt.lr = 1;
     if (PKV_W_TILE > 1 && a.cap_tiles == 0 && T > 0 &&

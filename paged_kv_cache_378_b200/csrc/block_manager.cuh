@@ -16,7 +16,9 @@
 //   - the k-th block taken, in writer order, is the free ring's entry at
 //     head + k (an exclusive scan of "takes a block" over the writers);
 //   - copy pairs are numbered by an exclusive scan of "copies".
-// One CTA of 1024 threads; writer i is handled by thread i mod 1024.
+// One CTA of 1024 threads; writer i is handled by thread i mod 1024.  All
+// reads and decisions come before the wait on the previous kernel, all writes
+// after it.
 //
 // An abort (free blocks short, an index out of range) changes no state and
 // leaves outputs that make a step queued behind it harmless: every slot -1,
@@ -78,16 +80,23 @@ __device__ __forceinline__ int bm_scan(int v, int* s_warp, int* total) {
 }
 
 __global__ void __launch_bounds__(BM_THREADS, 1) block_manager_kernel(const BmArgs a) {
-    // The tables, lengths and counts may still be read by the kernel before
-    // this one.  This kernel never releases its dependents early: the next
-    // attention launch reads the lengths before its own wait.
-    pdl_wait();
+    // Reads first, writes after the wait.  What this kernel reads (order,
+    // lengths, tables, counts, free ring and state) is written only by this
+    // kernel, which never releases its dependents early (so an earlier step
+    // has completed before this one starts), and by copies; so every read and
+    // decision runs before the wait, overlapping the tail of the kernel before
+    // it on the stream (an attention launch that still reads the tables), and
+    // every write comes after.  Not releasing early also lets the next
+    // attention launch read the new lengths before its own wait.
     __shared__ int s_tail[BM_MAX_SEQS];                 // tail block of writer i, -1: takes a new one
+    __shared__ int s_list[BM_MAX_SEQS];                 // writers whose tail is shared (any order)
     __shared__ int s_warp[33];
-    __shared__ int s_abort;
+    __shared__ int s_abort, s_nlist;
     const int N = a.num_seqs, B = a.block_size;
     const int tid = threadIdx.x;
-    if (tid == 0) s_abort = 0;
+    if (tid == 0) { s_abort = 0; s_nlist = 0; }
+    const int head = a.free_state[0], avail = a.free_state[1];
+    __syncthreads();
 
     // writer i = k * BM_THREADS + tid: one per thread for up to 1024 sequences
     int seq[BM_PER_THREAD], pos[BM_PER_THREAD], cnt[BM_PER_THREAD];
@@ -108,40 +117,47 @@ __global__ void __launch_bounds__(BM_THREADS, 1) block_manager_kernel(const BmAr
             if (tail < 0 || tail >= a.num_blocks) { raise_status(PKV_DEV_RANGE); atomicExch(&s_abort, 1); continue; }
             s_tail[i] = tail;
             cnt[k] = a.refcount[tail];
+            if (cnt[k] > 1) s_list[atomicAdd(&s_nlist, 1)] = i;
         }
     }
     __syncthreads();
 
-    // which writers take a block, which of them copy: only writers on a shared
-    // tail need their rank among earlier writers of the same block
-    int takes[BM_PER_THREAD], copies[BM_PER_THREAD];
+    // which writers take a block, which of them copy: a writer on a shared
+    // tail needs its rank among earlier writers of the same block, counted
+    // over the (usually short) list of writers on shared tails
+    int v[BM_PER_THREAD];                               // takes | copies << 16
+    const int nlist = s_nlist;
 #pragma unroll
     for (int k = 0; k < BM_PER_THREAD; ++k) {
         const int i = k * BM_THREADS + tid;
-        takes[k] = copies[k] = 0;
+        v[k] = 0;
         if (seq[k] < 0) continue;
         const int tail = s_tail[i];
         if (tail < 0) {
-            takes[k] = 1;
+            v[k] = 1;
         } else if (cnt[k] > 1) {
             int r = 0;                                  // earlier writers on the same tail
-            for (int j = 0; j < i && r < cnt[k] - 1; ++j) r += (s_tail[j] == tail);
-            if (cnt[k] - r > 1) takes[k] = copies[k] = 1;
+            for (int j = 0; j < nlist; ++j) {
+                const int w = s_list[j];
+                r += (w < i && s_tail[w] == tail);
+            }
+            if (cnt[k] - r > 1) v[k] = 1 | (1 << 16);
         }
     }
-    // exclusive scans in writer order, one round of BM_THREADS writers at a time
+    // one exclusive scan in writer order of both counts (each below 2^16),
+    // one round of BM_THREADS writers at a time
     int take_base[BM_PER_THREAD], copy_base[BM_PER_THREAD];
     int total_takes = 0, total_copies = 0;
 #pragma unroll
     for (int k = 0; k < BM_PER_THREAD; ++k) {
         if (k * BM_THREADS >= N) { take_base[k] = copy_base[k] = 0; continue; }   // uniform
-        int t, c;
-        take_base[k] = total_takes + bm_scan(takes[k], s_warp, &t);
-        copy_base[k] = total_copies + bm_scan(copies[k], s_warp, &c);
-        total_takes += t;
-        total_copies += c;
+        int t;
+        const int before = bm_scan(v[k], s_warp, &t);
+        take_base[k] = total_takes + (before & 0xFFFF);
+        copy_base[k] = total_copies + (before >> 16);
+        total_takes += t & 0xFFFF;
+        total_copies += t >> 16;
     }
-    const int head = a.free_state[0], avail = a.free_state[1];
     // the blocks the takers will get, checked before anything changes
     int newb[BM_PER_THREAD];
 #pragma unroll
@@ -149,13 +165,16 @@ __global__ void __launch_bounds__(BM_THREADS, 1) block_manager_kernel(const BmAr
     if (total_takes <= avail) {
 #pragma unroll
         for (int k = 0; k < BM_PER_THREAD; ++k) {
-            if (seq[k] < 0 || !takes[k]) continue;
+            if (seq[k] < 0 || !(v[k] & 1)) continue;
             newb[k] = a.free_ring[(head + take_base[k]) % a.num_blocks];
             if (newb[k] < 0 || newb[k] >= a.num_blocks) { raise_status(PKV_DEV_RANGE); atomicExch(&s_abort, 1); }
         }
     }
     __syncthreads();
-    if (s_abort || total_takes > avail) {
+    const bool abort = s_abort || total_takes > avail;
+
+    pdl_wait();                                         // the kernel before this one has finished
+    if (abort) {
         // Change nothing, and say so to whatever is queued behind this step:
         // no slot (kv_append skips slot -1), no copy pair, and per sequence
         // the marker that makes the fused append + attention append nothing.
@@ -167,26 +186,27 @@ __global__ void __launch_bounds__(BM_THREADS, 1) block_manager_kernel(const BmAr
         if (tid == 0) *a.num_pairs = 0;
         return;
     }
-    __syncthreads();                                    // every count read before any is changed
 
 #pragma unroll
     for (int k = 0; k < BM_PER_THREAD; ++k) {
         if (seq[k] < 0) continue;
         const int s = seq[k], p = pos[k];
+        const int tail = s_tail[k * BM_THREADS + tid];
+        const bool copies = (v[k] >> 16) != 0;
         int32_t* entry = a.block_tables + (size_t)s * a.max_blocks + p / B;
-        if (takes[k]) {
-            const int nb = newb[k];
-            a.refcount[nb] = 1;
-            if (copies[k]) {
-                const int tail = s_tail[k * BM_THREADS + tid];
+        int blk = tail;
+        if (v[k] & 1) {
+            blk = newb[k];
+            a.refcount[blk] = 1;
+            if (copies) {
                 a.copy_pairs[2 * copy_base[k]] = tail;
-                a.copy_pairs[2 * copy_base[k] + 1] = nb;
+                a.copy_pairs[2 * copy_base[k] + 1] = blk;
                 atomicSub(a.refcount + tail, 1);
             }
-            *entry = nb;
+            *entry = blk;
         }
-        if (a.cow_src) a.cow_src[s] = copies[k] ? s_tail[k * BM_THREADS + tid] : -1;
-        a.slot_mapping[s] = (int64_t)(*entry) * B + p % B;
+        if (a.cow_src) a.cow_src[s] = copies ? tail : -1;
+        a.slot_mapping[s] = (int64_t)blk * B + p % B;
         a.seq_lens[s] = p + 1;
     }
     if (tid == 0) {
