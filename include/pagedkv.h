@@ -271,6 +271,36 @@ int pkv_block_manager_step(const pkv_block_state_t* state, int num_seqs,
                            void* stream);
 
 /*
+ * pkv_block_manager_release -- finished requests give their blocks back, on
+ * the device.
+ *
+ * Defines ("Infra: PagedAttention", "按 Block 分配": a finished request drops
+ * its references; ithelp article 10405755, "手動畫一次 block table": when the
+ * request ends its blocks return to the pool): for each row of `seqs`, in the
+ * given order, each block of the row's table, in table order, loses one
+ * reference; a block whose count reaches zero is appended to the free ring
+ * after the blocks already free, in that order of drops (head unchanged,
+ * count grows).  The row's length becomes 0 and its table entries -1, so the
+ * row can serve a new request: the next pkv_block_manager_step gives it a
+ * fresh block for its first token.
+ *
+ *   state        as for pkv_block_manager_step, num_seqs rows
+ *   seqs         device int32 [num_release]: the rows to release, distinct
+ *   num_release  0..num_seqs
+ * The state must be consistent (each count equal to the number of table
+ * entries, over all rows, that name the block).  Errors: PKV_ERR_SHAPE,
+ * PKV_ERR_NULL, PKV_ERR_UNSUPPORTED (num_seqs > 4096), PKV_ERR_CUDA.  On the
+ * device, a row out of range or named twice, a length above the table, a
+ * block id out of range, more drops on a block than its count, or more than
+ * 8192 drops on shared blocks in one call set PKV_DEV_RANGE / PKV_DEV_LENGTH
+ * and change nothing.  The kernel waits for the kernel before it on the
+ * stream before reading anything and does not release its dependents early.
+ */
+int pkv_block_manager_release(const pkv_block_state_t* state, int num_seqs,
+                              int max_blocks_per_seq, int num_blocks, int block_size,
+                              const int32_t* seqs, int num_release, void* stream);
+
+/*
  * pkv_attention_workspace_bytes -- bytes of workspace pkv_paged_decode_attention
  * needs for these sizes on the current device: the tile prefix per sequence
  * (batches over 768 sequences; smaller ones keep it in shared memory), the

@@ -28,7 +28,8 @@ from ._lib import PkvBlockState, PkvCache
 
 __all__ = [
     "PagedKVError", "kv_append", "block_copy", "paged_decode_attention",
-    "append_paged_decode_attention", "BlockState", "block_manager_step", "swap_blocks",
+    "append_paged_decode_attention", "BlockState", "block_manager_step", "block_manager_release",
+    "swap_blocks",
     "SWAP_OUT", "SWAP_IN", "prefix_block_hashes",
     "attention_workspace_bytes", "partition_tokens", "make_workspace",
     "get_device_status", "set_wait_limit_ns", "workspace_init", "library", "DEV_RANGE",
@@ -265,6 +266,24 @@ def block_manager_step(state, block_size, order=None, stream=None, with_cow_src=
     if with_cow_src:
         return slots, pairs[:N], npairs, cow[:N]
     return slots, pairs[:N], npairs
+
+
+def block_manager_release(state, block_size, seqs, stream=None):
+    """Finished requests give their blocks back, on the device: ``seqs`` (int32
+    ``[k]``, distinct rows) in order, each row's blocks in table order, lose a
+    reference; blocks left with none join the free ring in that order; the
+    rows' lengths become 0 and their tables -1.  Updates ``state`` in place."""
+    dev = state.block_tables.device
+    N, maxb = state.block_tables.shape
+    nb = state.refcount.shape[0]
+    _need(seqs, "seqs", torch.int32, dev)
+    if seqs.dim() != 1:
+        raise ValueError("seqs must be [k]")
+    c = state._c()
+    rc = library().pkv_block_manager_release(
+        ctypes.byref(c), N, maxb, nb, int(block_size), seqs.data_ptr() if seqs.numel() else None,
+        int(seqs.numel()), _stream(dev, stream))
+    _check(rc, "block_manager_release")
 
 
 def attention_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,

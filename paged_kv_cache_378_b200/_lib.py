@@ -49,6 +49,9 @@ SIGNATURES = {
         ctypes.POINTER(PkvBlockState), ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
         ctypes.c_void_p]),
+    "pkv_block_manager_release": (ctypes.c_int, [
+        ctypes.POINTER(PkvBlockState), ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "pkv_attention_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 7),
     "pkv_partition_tokens": (ctypes.c_int, [ctypes.c_int] * 6),
     "pkv_workspace_init": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),

@@ -216,4 +216,164 @@ __global__ void __launch_bounds__(BM_THREADS, 1) block_manager_kernel(const BmAr
     }
 }
 
+// ---- release: finished requests give their blocks back ---------------------------
+//
+// What it computes ("Infra: PagedAttention", section 按 Block 分配: a finished
+// request drops its references; ithelp article 10405755, section 手動畫一次
+// block table: when the request ends its blocks return to the pool): for each
+// released sequence in the given order, each block of its table in table
+// order loses one reference, and a block whose count reaches zero is appended
+// to the free ring, after the blocks already free, in that order of drops.
+// The sequence's length becomes 0 and its table row -1.
+//
+// The order of drops is made without a serial walk: drop e (release r, table
+// entry j, numbered by a scan of the released sequences' block counts) on a
+// block of count c frees it exactly when it is the c-th drop on that block,
+// i.e. when r_e = c - 1 earlier drops hit the same block.  Unshared blocks
+// (c = 1) are freed by their one drop; drops on shared blocks list themselves
+// in shared memory and count the earlier ones there.  Ring positions are an
+// exclusive scan of "frees" in drop order.  Every check comes before any
+// write, so an invalid request changes nothing.
+constexpr int BR_MAX_SHARED = 8192;                  // drops on shared blocks one call can take
+
+struct BrArgs {
+    int32_t* block_tables;      // [N][max_blocks]
+    int32_t* seq_lens;          // [N]
+    int32_t* refcount;          // [num_blocks]
+    int32_t* free_ring;         // [num_blocks]
+    int32_t* free_state;        // [2] head, count
+    const int32_t* seqs;        // [num_release] rows to release, distinct
+    int num_seqs;
+    int num_release;
+    int max_blocks;
+    int num_blocks;
+    int block_size;
+};
+
+struct BrShared {
+    int off[BM_MAX_SEQS + 1];                        // first drop of release r; off[n] = drops
+    unsigned seen[BM_MAX_SEQS / 32];                 // rows named so far (duplicates abort)
+    int nlist;
+    int abort;
+    int warp[33];
+    int list_e[BR_MAX_SHARED], list_b[BR_MAX_SHARED], list_c[BR_MAX_SHARED];
+};
+
+__global__ void __launch_bounds__(BM_THREADS, 1) block_release_kernel(const BrArgs a) {
+    extern __shared__ unsigned char br_smem_raw[];
+    BrShared& sh = *reinterpret_cast<BrShared*>(br_smem_raw);
+    const int tid = threadIdx.x;
+    const int n = a.num_release, B = a.block_size;
+    pdl_wait();                                       // earlier steps' writes have landed
+    for (int i = tid; i < BM_MAX_SEQS / 32; i += BM_THREADS) sh.seen[i] = 0u;
+    if (tid == 0) { sh.nlist = 0; sh.abort = 0; }
+    __syncthreads();
+
+    // the released rows, their block counts and the drop numbering
+    int carry = 0;
+    for (int base = 0; base < n; base += BM_THREADS) {   // uniform trip count
+        const int r = base + tid;
+        int nb = 0;
+        if (r < n) {
+            const int s = a.seqs[r];
+            if (s < 0 || s >= a.num_seqs) {
+                raise_status(PKV_DEV_RANGE); atomicExch(&sh.abort, 1);
+            } else if (atomicOr(&sh.seen[s >> 5], 1u << (s & 31)) & (1u << (s & 31))) {
+                raise_status(PKV_DEV_RANGE); atomicExch(&sh.abort, 1);   // named twice
+            } else {
+                const int len = a.seq_lens[s];
+                nb = len > 0 ? (len + B - 1) / B : 0;
+                if (len < 0 || nb > a.max_blocks) {
+                    raise_status(PKV_DEV_LENGTH); atomicExch(&sh.abort, 1); nb = 0;
+                }
+            }
+        }
+        int tot;
+        const int before = bm_scan(nb, sh.warp, &tot);
+        if (r < n) sh.off[r] = carry + before;
+        carry += tot;
+    }
+    if (tid == 0) sh.off[n] = carry;
+    __syncthreads();
+    const int E = carry;
+    // drop e -> (release r, table entry j): the last r with off[r] <= e
+    auto locate = [&](int e, int& r, int& j) {
+        int lo = 0, hi = n - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sh.off[mid] <= e) lo = mid; else hi = mid - 1;
+        }
+        r = lo;
+        j = e - sh.off[lo];
+    };
+    auto block_of = [&](int e, int& blk) -> bool {
+        int r, j;
+        locate(e, r, j);
+        blk = a.block_tables[(size_t)a.seqs[r] * a.max_blocks + j];
+        return blk >= 0 && blk < a.num_blocks;
+    };
+
+    // checks, and the list of drops on shared blocks
+    if (!sh.abort) {
+        for (int e = tid; e < E; e += BM_THREADS) {
+            int blk;
+            if (!block_of(e, blk)) { raise_status(PKV_DEV_RANGE); atomicExch(&sh.abort, 1); continue; }
+            const int c = a.refcount[blk];
+            if (c <= 0) { raise_status(PKV_DEV_RANGE); atomicExch(&sh.abort, 1); continue; }
+            if (c > 1) {
+                const int k = atomicAdd(&sh.nlist, 1);
+                if (k < BR_MAX_SHARED) { sh.list_e[k] = e; sh.list_b[k] = blk; sh.list_c[k] = c; }
+                else { raise_status(PKV_DEV_RANGE); atomicExch(&sh.abort, 1); }
+            }
+        }
+    }
+    __syncthreads();
+    if (sh.abort) return;                             // nothing written
+    const int nlist = sh.nlist;
+    // drops on a block beyond its count: a count that would fall below zero
+    for (int k = tid; k < nlist; k += BM_THREADS) {
+        int r = 0;
+        for (int q = 0; q < nlist; ++q) r += (sh.list_b[q] == sh.list_b[k] && sh.list_e[q] < sh.list_e[k]);
+        if (r >= sh.list_c[k]) { raise_status(PKV_DEV_RANGE); atomicExch(&sh.abort, 1); }
+    }
+    __syncthreads();
+    if (sh.abort) return;
+
+    // which drops free their block, and where it goes in the ring (counts not yet changed)
+    const int head = a.free_state[0], avail = a.free_state[1];
+    int freed = 0;
+    for (int base = 0; base < E; base += BM_THREADS) {   // uniform trip count
+        const int e = base + tid;
+        int frees = 0, blk = -1;
+        if (e < E) {
+            block_of(e, blk);
+            const int c = a.refcount[blk];
+            if (c == 1) {
+                frees = 1;
+            } else {
+                int r = 0;
+                for (int q = 0; q < nlist; ++q) r += (sh.list_b[q] == blk && sh.list_e[q] < e);
+                frees = r == c - 1;
+            }
+        }
+        int tot;
+        const int before = bm_scan(frees, sh.warp, &tot);
+        if (frees) a.free_ring[(head + avail + freed + before) % a.num_blocks] = blk;
+        freed += tot;
+    }
+    __syncthreads();                                  // every count read before any changes
+    for (int e = tid; e < E; e += BM_THREADS) {
+        int blk;
+        block_of(e, blk);
+        atomicSub(a.refcount + blk, 1);
+    }
+    __syncthreads();                                  // every table entry read before any is reset
+    for (int r = 0; r < n; ++r) {
+        const int s = a.seqs[r];
+        for (int j = tid; j < a.max_blocks; j += BM_THREADS) a.block_tables[(size_t)s * a.max_blocks + j] = -1;
+        if (tid == 0) a.seq_lens[s] = 0;
+    }
+    if (tid == 0) a.free_state[1] = avail + freed;
+}
+
 }  // namespace pkv

@@ -552,6 +552,43 @@ int pkv_block_manager_step(const pkv_block_state_t* st, int num_seqs, int max_bl
                       (cudaStream_t)stream, a);
 }
 
+int pkv_block_manager_release(const pkv_block_state_t* st, int num_seqs, int max_blocks_per_seq,
+                              int num_blocks, int block_size, const int32_t* seqs, int num_release,
+                              void* stream) {
+    if (!st) return PKV_ERR_NULL;
+    if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || block_size <= 0 ||
+        num_release < 0 || num_release > num_seqs)
+        return PKV_ERR_SHAPE;
+    if (num_seqs > pkv::BM_MAX_SEQS) return PKV_ERR_UNSUPPORTED;
+    if (num_release == 0) return PKV_OK;
+    if (!st->block_tables || !st->seq_lens || !st->refcount || !st->free_ring || !st->free_state ||
+        !seqs)
+        return PKV_ERR_NULL;
+    static bool configured[kMaxDevices] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+    if (!configured[dev]) {
+        if (cudaFuncSetAttribute(pkv::block_release_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(pkv::BrShared)) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        configured[dev] = true;
+    }
+    pkv::BrArgs a;
+    a.block_tables = st->block_tables;
+    a.seq_lens = st->seq_lens;
+    a.refcount = st->refcount;
+    a.free_ring = st->free_ring;
+    a.free_state = st->free_state;
+    a.seqs = seqs;
+    a.num_seqs = num_seqs;
+    a.num_release = num_release;
+    a.max_blocks = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
+    a.block_size = block_size;
+    return launch_pdl(pkv::block_release_kernel, dim3(1), dim3(pkv::BM_THREADS), sizeof(pkv::BrShared),
+                      (cudaStream_t)stream, a);
+}
+
 int pkv_partition_tokens(int num_seqs, int num_kv_heads, int head_dim, int max_blocks_per_seq,
                          int block_size, int requested) {
     if (!supported_head_dim(head_dim) || num_seqs < 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0)

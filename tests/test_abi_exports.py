@@ -128,6 +128,15 @@ def test_host_argument_checks_before_launch():
     assert bm(P(st), 0, 8, 64, 16, None, 16, 16, 16, None, None) == 0
     assert bm(P(st), 4, 8, 64, 16, None, None, 16, 16, None, None) == -1
     assert bm(P(_lib.PkvBlockState(16, 0, 16, 16, 16)), 4, 8, 64, 16, None, 16, 16, 16, None, None) == -1
+    # device release: state and rows required, at most num_seqs rows, at most 4096 sequences
+    rel = lib.pkv_block_manager_release
+    assert rel(None, 4, 8, 64, 16, 16, 2, None) == -1
+    assert rel(P(st), 4, 8, 64, 16, 16, 5, None) == -2
+    assert rel(P(st), 4, 8, 64, 16, 16, -1, None) == -2
+    assert rel(P(st), 4097, 8, 64, 16, 16, 2, None) == -5
+    assert rel(P(st), 4, 8, 64, 16, None, 0, None) == 0
+    assert rel(P(st), 4, 8, 64, 16, None, 2, None) == -1
+    assert rel(P(_lib.PkvBlockState(16, 16, 0, 16, 16)), 4, 8, 64, 16, 16, 2, None) == -1
 
 
 def test_workspace_and_partition_sizes():
