@@ -697,6 +697,66 @@ paged_attention_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 stored = true;
             }
             if (lane == 0) st_cg(reinterpret_cast<int*>(ticket), 0);   // ready for the next launch
+            if (G < 8 && D == 64) {
+                // Fetch rounds: every lane loads, not only the lanes of the G
+                // rows; lane row g_row takes element e0 + g_row / G, row
+                // g_row % G, so one round trip brings 8 / G elements.  The fold
+                // takes them in element order through shuffles: the same
+                // arithmetic, in the same order, as the path below.  (At head_dim
+                // 128 the extra registers spill and cost more than they save.)
+                constexpr int S = 8 / G;
+                const int k_lane = g_row / G, r_lane = g_row % G;
+                if (mine != first && !stored) store_state(slot_of(mine));
+                __syncwarp();
+                bool acc = mine == first;                   // the state holds element `first`
+                float2 v[D / 8], mz = make_float2(0.f, 0.f);
+                for (long long e0 = acc ? first + 1 : first; e0 <= last; e0 += S) {
+                    const long long el = e0 + k_lane;
+                    if (el <= last) {
+                        const size_t pr = slot_of(el) - g_row + r_lane;
+                        const float* po = a.part_o + pr * D + 2 * c4;
+#pragma unroll
+                        for (int n = 0; n < D / 8; ++n) v[n] = ld_cg(reinterpret_cast<const float2*>(po + 8 * n));
+                        mz = ld_cg(a.part_mz + pr);
+                    }
+#pragma unroll
+                    for (int k = 0; k < S; ++k) {
+                        if (e0 + k > last) break;
+                        const int src = lane + 4 * G * k;       // the lane holding this row of element e0 + k
+                        auto take = [&](float2 x) -> float2 {
+                            return k == 0 ? x : make_float2(__shfl_sync(FULL, x.x, src), __shfl_sync(FULL, x.y, src));
+                        };
+                        const float2 wz = take(mz);
+                        if (!acc) {
+#pragma unroll
+                            for (int n = 0; n < D / 8; ++n) {
+                                const float2 w = take(v[n]);
+                                ws.o[n][0] = w.x;
+                                ws.o[n][1] = w.y;
+                            }
+                            M = wz.x;
+                            Z = wz.y;
+                            acc = true;
+                            continue;
+                        }
+                        const float mx = fmaxf(M, wz.x);
+                        const float ca = fast_exp2(M - mx), cb = fast_exp2(wz.x - mx);
+                        if (g_row < G) {
+                            Z = fmaf(cb, wz.y, Z * ca);
+                            M = mx;
+                        }
+#pragma unroll
+                        for (int n = 0; n < D / 8; ++n) {
+                            const float2 w = take(v[n]);
+                            if (g_row < G) {
+                                ws.o[n][0] = fmaf(cb, w.x, ws.o[n][0] * ca);
+                                ws.o[n][1] = fmaf(cb, w.y, ws.o[n][1] * ca);
+                            }
+                        }
+                    }
+                }
+                return true;
+            }
             if (mine != first) {                            // the fold starts from the first element
                 if (!stored) store_state(slot_of(mine));
                 __syncwarp();
