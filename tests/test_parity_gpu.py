@@ -166,18 +166,20 @@ def test_shape_sweep_with_split_partitions(D, G, B):
 
 
 @pytest.mark.parametrize("D", [64, 128])
-def test_many_pieces_two_level_merge(D):
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_many_pieces_two_level_merge(D, G):
     # one tile per range: a 4096-token sequence is 128 (d 64) or 256 (d 128)
-    # pieces per (sequence, kv head), merged in groups of ranges and then groups
-    spec = WorkloadSpec(key="custom", title="custom", num_layers=1, num_seqs=3, num_q_heads=8,
-                        num_kv_heads=2, head_dim=D, block_size=16, seed=7 + D,
+    # pieces per (sequence, kv head), merged in groups of ranges and then groups;
+    # at d 64 a merge fetches 8 / G pieces per round trip (G = 8: one)
+    spec = WorkloadSpec(key="custom", title="custom", num_layers=1, num_seqs=3, num_q_heads=2 * G,
+                        num_kv_heads=2, head_dim=D, block_size=16, seed=7 + D + G,
                         lengths="fixed:4096,1000,37")
     w = make_workload(spec)
     ref = _oracle_attention(w, 0)
     tile = 32 if D == 64 else 16
     outs = gpu_step(pkv, w, device_inputs(w), partition_tokens=tile)
     _assert_no_device_error()
-    assert_close(f64(outs[0]), ref, f"D={D} one tile per range")
+    assert_close(f64(outs[0]), ref, f"D={D} G={G} one tile per range")
     again = gpu_step(pkv, w, device_inputs(w), partition_tokens=tile)[0]
     assert torch.equal(outs[0].view(torch.int16), again.view(torch.int16))
 
