@@ -182,6 +182,24 @@ def test_copy_on_write_many_sharers():
     assert bm2.take_copy_pairs() == []
 
 
+def test_release_returns_shared_blocks_only_with_their_last_user():
+    # [PU] 按 Block 分配 / 共享前缀: a finished request drops its references; a
+    # block still referenced by another sequence stays out of the pool.  A and
+    # B share [P3, P0]; after A's write copied P0 -> P4, A ends: only P4 returns.
+    bm = op.BlockManager(8, 4, free_order=[3, 0, 4, 1, 2, 5, 6, 7])
+    bm.add_sequence("A", 6)
+    bm.fork("A", "B")
+    bm.append_slot("A")
+    assert bm.tables["A"] == [3, 4] and bm.tables["B"] == [3, 0]
+    free_before = list(bm.free)
+    bm.free_sequence("A")
+    assert list(bm.free) == free_before + [4]
+    assert bm.refcount[3] == 1 and bm.refcount[0] == 1
+    bm.free_sequence("B")
+    assert list(bm.free) == free_before + [4, 3, 0]
+    assert all(c == 0 for c in bm.refcount)
+
+
 def test_block_manager_exhaustion_and_release():
     bm = op.BlockManager(num_blocks=3, block_size=2)
     bm.add_sequence("x", 6)
