@@ -1165,6 +1165,9 @@ def main():
     # A spin kernel ahead of the region keeps the GPU busy while the host
     # enqueues the steps, so the events time the device, not the host's
     # first enqueue latency (a short region would otherwise include it).
+    # NVTX ranges mark the phases for a profiler's timeline (one push and
+    # pop per phase, none per launch)
+    torch.cuda.nvtx.range_push("timed steps")
     torch.cuda._sleep(SPIN_CYCLES)
     t_start.record(gs.stream)
     nl = spec.num_layers
@@ -1176,6 +1179,7 @@ def main():
         else:
             fast(i)
     t_end.record(gs.stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize(device)
     wall1 = time.time()
     if dist is not None:
@@ -1204,7 +1208,8 @@ def main():
         sampling = f"attention bracketed on every {EVENT_EVERY}th timed step"
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
     # per-launch distribution from a separate untimed pass (every launch alone)
-    stats = launch_stats(gs, max(50, min(500, args.steps)), args.steps + 10**6)
+    with torch.cuda.nvtx.range("per-launch statistics"):
+        stats = launch_stats(gs, max(50, min(500, args.steps)), args.steps + 10**6)
 
     # totals over ranks: device time is the max, work is the sum
     ms_max, bytes_total, seqs_total = combine_over_ranks(
@@ -1214,7 +1219,8 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e_ms, h2d, d2h, ncpu = e2e_run(pkv, w, gs, args.e2e_steps, device)
+        with torch.cuda.nvtx.range("end to end"):
+            e_ms, h2d, d2h, ncpu = e2e_run(pkv, w, gs, args.e2e_steps, device)
         e_ms = combine_over_ranks(dist, e_ms, 0, 0, device)[0]
         e2e = {"value": bytes_total / (e_ms * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
@@ -1224,6 +1230,7 @@ def main():
 
     extras = {}
     if not args.no_extras:
+        torch.cuda.nvtx.range_push("rows beyond attention")
         bm_us = block_manager_timing(pkv, w, device) if w.num_seqs <= 4096 else None
         bm_chain = (block_manager_chained_timing(pkv, w, gs, device)
                     if bm_us is not None and spec.num_layers == 1 else None)
@@ -1242,6 +1249,7 @@ def main():
                                 "step between them (it reads and decides before its wait on the "
                                 "previous launch, so only its writes and the next launch's start "
                                 "are added)"})
+        torch.cuda.nvtx.range_pop()
 
     peak, peak_kind = load_peak()
     alg = algorithmic_bytes(w, spec, B, gs, unique_bytes)
@@ -1258,8 +1266,9 @@ def main():
         per_config = []
         for key, bs, p in PER_CONFIG:
             sp = get_spec(key)
-            per_config.append(measure_config(pkv, key, bs, sp.partition_tokens if p < 0 else p,
-                                             device, sampler, peak, peak_kind))
+            with torch.cuda.nvtx.range(f"config {key} B={bs} partition={p}"):
+                per_config.append(measure_config(pkv, key, bs, sp.partition_tokens if p < 0 else p,
+                                                 device, sampler, peak, peak_kind))
     sampler.stop()
 
     # the oracle on the host cores last: a spawned pool, so starting it after
